@@ -1,0 +1,242 @@
+"""Float64 CPU oracle for attention states over sequence partitions.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may use it.  It shares no code with
+the CUDA path; both sides receive the same inputs from the seeded generators.
+
+It is a plain restatement of what DiTango ("DiTango: Cost-Effective Parallel
+Diffusion Generation with Selective Attention State Reuse", arXiv 2607.15650)
+computes, as summarised on its pith.science review page:
+
+* attention state (section "What carries the argument"): for a query row and
+  a KV partition j, AS(j) = (OUT(j), LSE(j)), the partial attention output of
+  the keys of j and the log-sum-exp of their scores;
+* composition (Axiom & Free-Parameter Ledger, Eq. 1-2, "standard result from
+  FlashAttention/FlashInfer"): states compose associatively and commutatively
+  by LSE weighting;
+* selective reuse (Core claim; Referee Report, Summary): at a step t the query
+  partition i computes fresh states for some KV partitions and reuses cached
+  states from an earlier step for the others; the final output is the
+  composition of both kinds.
+
+Readings where the page is silent (each is listed in the design notes):
+OUT is the *normalised* partial output; logs are natural; the LSE includes the
+softmax scale; attention is bidirectional with no mask or bias; partitions are
+contiguous, equal and in token order; the empty state is (OUT=0, LSE=-inf); a
+plan entry is 0=reuse, 1=fresh, 2=fresh and refresh the cached entry; hit is 1
+exactly for reused pairs and age = t - t_c for them (0 otherwise).
+
+Every pin of this module lives in ``tests/test_oracle.py``.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+PLAN_REUSE = 0
+PLAN_FRESH = 1
+PLAN_FRESH_STORE = 2
+
+
+class CacheMiss(Exception):
+    """A plan reuses a pair whose cache entry has never been written."""
+
+
+class PlanError(Exception):
+    """A plan matrix holds a value other than 0, 1 or 2, or has a wrong shape."""
+
+
+# ---------------------------------------------------------------------------
+# the attention state of one KV partition
+# ---------------------------------------------------------------------------
+
+def attention_state(q, k, v, scale):
+    """AS = (OUT, LSE) of the query rows ``q`` against the keys ``k``/``v``.
+
+    For a query row q_r: s_m = scale * <q_r, k_m> over the keys m of the
+    partition, LSE = ln sum_m exp(s_m), OUT = sum_m exp(s_m - LSE) * v_m.
+    Shapes: q [..., nq, d], k and v [..., nk, d]; returns OUT [..., nq, d] and
+    LSE [..., nq], float64.  With no keys the state is the empty state.
+    (DiTango review, "What carries the argument": AS_t(i) = (OUT_t(i), LSE_t(i)).)
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if k.shape[-2] == 0:
+        return empty_state(q.shape[:-1], v.shape[-1])
+    s = scale * (q @ np.swapaxes(k, -1, -2))            # [..., nq, nk]
+    m = s.max(axis=-1, keepdims=True)                     # shift for exp range only
+    e = np.exp(s - m)
+    l = e.sum(axis=-1, keepdims=True)
+    lse = (m + np.log(l))[..., 0]
+    out = (e @ v) / l
+    return out, lse
+
+
+def empty_state(row_shape, d):
+    """The neutral element of composition: OUT = 0, LSE = -inf."""
+    return np.zeros(tuple(row_shape) + (d,)), np.full(tuple(row_shape), -np.inf)
+
+
+# ---------------------------------------------------------------------------
+# composition (DiTango review, Axiom & Free-Parameter Ledger, Eq. 1-2)
+# ---------------------------------------------------------------------------
+
+def compose_pair(a, b):
+    """Compose two states: LSE = ln(e^{LSE_a} + e^{LSE_b}),
+    OUT = e^{LSE_a - LSE} OUT_a + e^{LSE_b - LSE} OUT_b.  Rows where both
+    states are empty stay empty."""
+    oa, la = a
+    ob, lb = b
+    m = np.maximum(la, lb)
+    safe_m = np.where(np.isfinite(m), m, 0.0)
+    ea = np.exp(la - safe_m)
+    eb = np.exp(lb - safe_m)
+    tot = ea + eb
+    lse = np.where(tot > 0, safe_m + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    wa = np.where(tot > 0, ea / np.where(tot > 0, tot, 1.0), 0.0)
+    wb = np.where(tot > 0, eb / np.where(tot > 0, tot, 1.0), 0.0)
+    out = wa[..., None] * oa + wb[..., None] * ob
+    return out, lse
+
+
+def compose(states):
+    """Compose any number of states in one pass (the N-ary form of the binary
+    rule; equal to any tree of ``compose_pair`` because composition is
+    associative and commutative).  ``states`` is a non-empty sequence of
+    (OUT, LSE) with matching shapes."""
+    states = list(states)
+    outs = np.stack([np.asarray(o, dtype=np.float64) for o, _ in states])  # [N, ..., d]
+    lses = np.stack([np.asarray(l, dtype=np.float64) for _, l in states])  # [N, ...]
+    m = lses.max(axis=0)
+    safe_m = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lses - safe_m)                                              # [N, ...]
+    tot = w.sum(axis=0)
+    nz = tot > 0
+    lse = np.where(nz, safe_m + np.log(np.where(nz, tot, 1.0)), -np.inf)
+    coef = np.where(nz, w / np.where(nz, tot, 1.0), 0.0)
+    out = (coef[..., None] * outs).sum(axis=0)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# partitions
+# ---------------------------------------------------------------------------
+
+def partition_bounds(S, P):
+    """Contiguous equal partitions in token order: j covers [j*S/P, (j+1)*S/P)."""
+    if P <= 0 or S % P != 0:
+        raise ValueError("S must be a positive multiple of P")
+    n = S // P
+    return [(j * n, (j + 1) * n) for j in range(P)]
+
+
+def partition_states(q, k, v, scale, P):
+    """States of the query rows ``q`` [B,H,nq,d] against every KV partition of
+    ``k``/``v`` [B,H,S,d]."""
+    S = k.shape[-2]
+    return [attention_state(q, k[..., a:b, :], v[..., a:b, :], scale)
+            for a, b in partition_bounds(S, P)]
+
+
+def full_attention(q, k, v, scale):
+    """Plain softmax attention over all keys, returned as a state."""
+    return attention_state(q, k, v, scale)
+
+
+# ---------------------------------------------------------------------------
+# plan resolution and the state cache
+# ---------------------------------------------------------------------------
+
+def resolve_plan(plan, t_c, t):
+    """Check a plan against the cache timestamps and derive hit and age.
+
+    plan [P,P] uint8 (row i = query partition, column j = KV partition), t_c
+    [P,P] int (step of the entry's last write, -1 = never written), t the
+    current step.  hit[i,j] = 1 for reused pairs, else 0; age[i,j] = t - t_c
+    for reused pairs, else 0.  A reuse of a never-written entry raises
+    CacheMiss; any other value than 0/1/2 raises PlanError.
+    """
+    plan = np.asarray(plan)
+    t_c = np.asarray(t_c)
+    P = plan.shape[0]
+    if plan.ndim != 2 or plan.shape != (P, P) or t_c.shape != (P, P):
+        raise PlanError("plan and t_c must both be [P, P]")
+    hit = np.zeros((P, P), dtype=np.uint8)
+    age = np.zeros((P, P), dtype=np.int32)
+    for i in range(P):
+        for j in range(P):
+            c = int(plan[i, j])
+            if c not in (PLAN_REUSE, PLAN_FRESH, PLAN_FRESH_STORE):
+                raise PlanError(f"plan[{i},{j}] = {c}")
+            if c == PLAN_REUSE:
+                if t_c[i, j] < 0:
+                    raise CacheMiss(f"pair ({i},{j}) reused before any store")
+                hit[i, j] = 1
+                age[i, j] = t - int(t_c[i, j])
+    return hit, age
+
+
+class StateCache:
+    """One cached state per (query partition i, KV partition j), for the query
+    rows the oracle evaluates, plus the step t_c of each entry's last write."""
+
+    def __init__(self, P):
+        self.P = P
+        self.t_c = np.full((P, P), -1, dtype=np.int64)
+        self.entry = {}
+
+
+def step(cache, q, k, v, plan, t, scale, rows=None):
+    """One denoising step's attention under a compute/reuse plan.
+
+    final(i) = compose({AS_t(i,j) : plan[i,j] fresh} U {C(i,j) : plan[i,j] = reuse}),
+    then C(i,j) <- AS_t(i,j) and t_c(i,j) <- t for plan[i,j] = fresh-and-store.
+    (DiTango review: Core claim and Referee Report Summary -- fresh states for
+    near partitions, cached composed states from earlier steps for far ones.)
+
+    q, k, v: [B,H,S,d].  ``rows``: sorted token indices of the query rows to
+    evaluate (default all); the same rows must be used at every step of one
+    cache.  Returns OUT [B,H,len(rows),d], LSE [B,H,len(rows)], hit, age.
+    The plan is validated (and CacheMiss raised) before anything changes.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    S = k.shape[-2]
+    P = cache.P
+    n = S // P
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    hit, age = resolve_plan(plan, cache.t_c, t)
+    B, H, _, d = q.shape
+    out = np.zeros((B, H, len(rows), d))
+    lse = np.zeros((B, H, len(rows)))
+    bounds = partition_bounds(S, P)
+    updates = []
+    for i in range(P):
+        sel = np.nonzero((rows >= i * n) & (rows < (i + 1) * n))[0]
+        if sel.size == 0:
+            continue
+        qi = q[:, :, rows[sel], :]
+        parts = []
+        for j, (a, b) in enumerate(bounds):
+            c = int(plan[i, j])
+            if c == PLAN_REUSE:
+                parts.append(cache.entry[(i, j)])
+            else:
+                st = attention_state(qi, k[..., a:b, :], v[..., a:b, :], scale)
+                parts.append(st)
+                if c == PLAN_FRESH_STORE:
+                    updates.append(((i, j), st))
+        o, l = compose(parts)
+        out[:, :, sel, :] = o
+        lse[:, :, sel] = l
+    for key, st in updates:
+        cache.entry[key] = st
+        cache.t_c[key] = t
+    return out, lse, hit, age
+
+
+def mse(a, b):
+    """Mean squared difference, used to report reuse error against full attention."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.mean((a - b) ** 2))

@@ -1,0 +1,33 @@
+"""Parser for the hand-computed plan fixtures under tests/golden/."""
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _matrix(lines, P, dtype):
+    return np.array([[int(x) for x in lines.pop(0).split()] for _ in range(P)], dtype=dtype)
+
+
+def load_plan_fixture(name="plan_4x4.txt"):
+    """Returns (P, [dict(step, plan, expect, hit, age)])."""
+    with open(os.path.join(GOLDEN, name)) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.lstrip().startswith("#")]
+    assert lines[0].startswith("P ")
+    P = int(lines.pop(0).split()[1])
+    cases = []
+    while lines:
+        head = lines.pop(0)
+        assert head.startswith("step "), head
+        case = {"step": int(head.split()[1])}
+        assert lines.pop(0) == "plan"
+        case["plan"] = _matrix(lines, P, np.uint8)
+        case["expect"] = lines.pop(0).split()[1]
+        if case["expect"] == "ok":
+            assert lines.pop(0) == "hit"
+            case["hit"] = _matrix(lines, P, np.uint8)
+            assert lines.pop(0) == "age"
+            case["age"] = _matrix(lines, P, np.int32)
+        cases.append(case)
+    return P, cases

@@ -1,0 +1,381 @@
+"""Pins for the float64 oracle, checked against things other than itself.
+
+Each ``pin_*`` takes the oracle module and raises on a mismatch.  The real
+oracle must pass every pin; each planted mistake in ``MUTANTS`` (a dropped
+term, a wrong sign, a transposed operand, a wrong index, wrong bookkeeping)
+must fail at least one pin, which shows the pins would notice it.
+
+What the pins compare against (none of it is the oracle's own formula):
+* pure-Python loops over math.exp on tiny inputs (brute force);
+* torch's scaled_dot_product_attention in float64 on the CPU (library);
+* scipy.special.logsumexp (library);
+* closed forms: zero query (uniform weights), identical keys, a single key,
+  equal-LSE halves, the empty state;
+* invariants the pages state: composition is associative and commutative
+  (DiTango review, Axiom & Free-Parameter Ledger, Eq. 1-2), composing the
+  states of all partitions gives full attention, one partition is plain
+  attention;
+* the hand-computed plan/cache fixture tests/golden/plan_4x4.txt;
+* reuse identities: cached states of KV partitions whose inputs did not move
+  are exact, so a reuse step then equals full attention over the mixed inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import as_oracle
+from tests._golden import load_plan_fixture
+
+TOL = 1e-11
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _sdpa(q, k, v, scale):
+    out = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), scale=scale)
+    return out.numpy()
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    finite = np.isfinite(b)
+    assert np.array_equal(np.isfinite(a), finite), f"{what}: finiteness differs"
+    assert np.array_equal(a[~finite], b[~finite]), f"{what}: infinities differ"
+    err = np.max(np.abs(a[finite] - b[finite])) if finite.any() else 0.0
+    assert err <= tol, f"{what}: max abs err {err}"
+
+
+# ---------------------------------------------------------------------------
+# pins
+# ---------------------------------------------------------------------------
+
+def pin_bruteforce_loops(o):
+    r = _rng(1)
+    nq, nk, d = 5, 9, 4
+    q, k, v = r.normal(size=(nq, d)), r.normal(size=(nk, d)), r.normal(size=(nk, d))
+    scale = 0.7
+    out, lse = o.attention_state(q, k, v, scale)
+    for a in range(nq):
+        scores = [scale * sum(q[a][c] * k[m][c] for c in range(d)) for m in range(nk)]
+        z = sum(math.exp(s) for s in scores)
+        _close(lse[a], math.log(z), 1e-12, "bruteforce LSE")
+        for c in range(d):
+            ref = sum(math.exp(scores[m]) / z * v[m][c] for m in range(nk))
+            _close(out[a][c], ref, 1e-12, "bruteforce OUT")
+
+
+def pin_torch_sdpa_full(o):
+    r = _rng(2)
+    B, H, S, d, P = 2, 3, 40, 16, 5
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    scale = 1 / math.sqrt(d)
+    ref = _sdpa(q, k, v, scale)
+    out, _ = o.compose(o.partition_states(q, k, v, scale, P))
+    _close(out, ref, TOL, "composed vs sdpa")
+    out1, _ = o.full_attention(q, k, v, scale)
+    _close(out1, ref, TOL, "full vs sdpa")
+
+
+def pin_scipy_lse(o):
+    r = _rng(3)
+    q, k, v = r.normal(size=(7, 8)), r.normal(size=(11, 8)), r.normal(size=(11, 8))
+    scale = 0.3
+    _, lse = o.attention_state(q, k, v, scale)
+    for a in range(7):
+        scores = np.array([scale * np.dot(q[a], k[m]) for m in range(11)])
+        _close(lse[a], scipy.special.logsumexp(scores), 1e-12, "lse vs scipy")
+
+
+def pin_closed_forms(o):
+    r = _rng(4)
+    nk, d = 13, 6
+    k, v = r.normal(size=(nk, d)), r.normal(size=(nk, d))
+    # zero query: uniform weights, LSE = ln nk
+    out, lse = o.attention_state(np.zeros((2, d)), k, v, 0.9)
+    _close(out, np.tile(v.mean(axis=0), (2, 1)), 1e-12, "zero query OUT")
+    _close(lse, np.full(2, math.log(nk)), 1e-12, "zero query LSE")
+    # identical keys: LSE = scale<q,k0> + ln nk, OUT = mean v
+    q = r.normal(size=(3, d))
+    k0 = r.normal(size=d)
+    out, lse = o.attention_state(q, np.tile(k0, (nk, 1)), v, 0.5)
+    _close(out, np.tile(v.mean(axis=0), (3, 1)), 1e-12, "equal keys OUT")
+    _close(lse, 0.5 * (q @ k0) + math.log(nk), 1e-12, "equal keys LSE")
+    # a single key: OUT = v0, LSE = score
+    out, lse = o.attention_state(q, k0[None, :], v[:1], 0.5)
+    _close(out, np.tile(v[0], (3, 1)), 1e-12, "single key OUT")
+    _close(lse, 0.5 * (q @ k0), 1e-12, "single key LSE")
+    # no keys: the empty state
+    out, lse = o.attention_state(q, np.zeros((0, d)), np.zeros((0, d)), 0.5)
+    assert np.all(out == 0) and np.all(lse == -np.inf)
+
+
+def pin_compose_closed(o):
+    r = _rng(5)
+    oa, ob, oc = (r.normal(size=(4, 3)) for _ in range(3))
+    L = r.normal(size=4)
+    for f in (lambda a, b: o.compose([a, b]), o.compose_pair):
+        out, lse = f((oa, L), (ob, L))
+        _close(lse, L + math.log(2), 1e-12, "equal halves LSE")
+        _close(out, (oa + ob) / 2, 1e-12, "equal halves OUT")
+        out, lse = f((oa, L), (ob, np.full(4, -np.inf)))
+        _close(lse, L, 1e-12, "with empty LSE")
+        _close(out, oa, 1e-12, "with empty OUT")
+        out, lse = f((oa, np.full(4, -np.inf)), (ob, np.full(4, -np.inf)))
+        assert np.all(lse == -np.inf) and np.all(out == 0) and not np.isnan(out).any()
+    out, lse = o.compose([(oa, L), (ob, L + math.log(2)), (oc, L + math.log(3))])
+    _close(lse, L + math.log(6), 1e-12, "1:2:3 LSE")
+    _close(out, (oa + 2 * ob + 3 * oc) / 6, 1e-12, "1:2:3 OUT")
+
+
+def pin_assoc_comm(o):
+    r = _rng(6)
+    n = 7
+    states = [(r.normal(size=(5, 4)), r.normal(size=5) * 3) for _ in range(n)]
+    ref_o, ref_l = o.compose(states)
+    for trial in range(6):
+        perm = r.permutation(n)
+        pool = [states[p] for p in perm]
+        while len(pool) > 1:
+            a = r.integers(len(pool) - 1)
+            merged = o.compose_pair(pool[a], pool[a + 1])
+            pool[a:a + 2] = [merged]
+        _close(pool[0][0], ref_o, TOL, "random tree OUT")
+        _close(pool[0][1], ref_l, TOL, "random tree LSE")
+        po, pl = o.compose([states[p] for p in perm])
+        _close(po, ref_o, TOL, "permuted OUT")
+        _close(pl, ref_l, TOL, "permuted LSE")
+
+
+def pin_split_invariance(o):
+    r = _rng(7)
+    nk, d = 37, 8
+    q, k, v = r.normal(size=(6, d)), r.normal(size=(nk, d)), r.normal(size=(nk, d))
+    whole_o, whole_l = o.attention_state(q, k, v, 0.4)
+    for trial in range(4):
+        cuts = np.sort(r.choice(np.arange(1, nk), size=r.integers(1, 6), replace=False))
+        edges = [0] + list(cuts) + [nk]
+        parts = [o.attention_state(q, k[a:b], v[a:b], 0.4) for a, b in zip(edges[:-1], edges[1:])]
+        po, pl = o.compose(parts)
+        _close(po, whole_o, TOL, "split OUT")
+        _close(pl, whole_l, TOL, "split LSE")
+
+
+def pin_single_partition(o):
+    r = _rng(8)
+    q, k, v = (r.normal(size=(1, 2, 24, 8)) for _ in range(3))
+    (out, _), = o.partition_states(q, k, v, 0.35, 1)
+    _close(out, _sdpa(q, k, v, 0.35), TOL, "P=1 vs sdpa")
+
+
+def pin_plan_golden(o):
+    P, cases = load_plan_fixture()
+    r = _rng(9)
+    S, d = 2 * P, 3
+    q, k, v = (r.normal(size=(1, 1, S, d)) for _ in range(3))
+    cache = o.StateCache(P)
+    for c in cases:
+        if c["expect"] == "cache_miss":
+            before = cache.t_c.copy()
+            with pytest.raises(o.CacheMiss):
+                o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
+            assert np.array_equal(cache.t_c, before), "cache changed on a miss"
+            continue
+        if c["expect"] == "invalid":
+            with pytest.raises(o.PlanError):
+                o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
+            continue
+        _, _, hit, age = o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
+        assert np.array_equal(hit, c["hit"]), f"hit at step {c['step']}"
+        assert np.array_equal(age, c["age"]), f"age at step {c['step']}"
+
+
+def _window_plans(P, w):
+    i = np.arange(P)[:, None]
+    j = np.arange(P)[None, :]
+    near = np.abs(i - j) <= w
+    anchor = np.where(near, o_FRESH, o_STORE).astype(np.uint8)
+    reuse = np.where(near, o_FRESH, o_REUSE).astype(np.uint8)
+    return anchor, reuse
+
+
+o_REUSE, o_FRESH, o_STORE = 0, 1, 2
+
+
+def pin_step_all_fresh(o):
+    r = _rng(10)
+    B, H, S, d, P = 1, 2, 48, 8, 6
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    cache = o.StateCache(P)
+    out, lse, hit, age = o.step(cache, q, k, v, np.ones((P, P), np.uint8), 0, 0.3)
+    _close(out, _sdpa(q, k, v, 0.3), TOL, "all fresh vs sdpa")
+    _close(lse, scipy.special.logsumexp(0.3 * np.einsum("bhqd,bhkd->bhqk", q, k), axis=-1),
+           TOL, "all fresh LSE vs scipy")
+    assert not hit.any() and not age.any()
+    assert (cache.t_c == -1).all(), "fresh (code 1) pairs must not be stored"
+
+
+def pin_step_reuse_identical(o):
+    r = _rng(11)
+    B, H, S, d, P = 1, 2, 64, 8, 8
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    anchor, reuse = _window_plans(P, 1)
+    cache = o.StateCache(P)
+    o.step(cache, q, k, v, anchor, 0, 0.3)
+    out, _, hit, age = o.step(cache, q, k, v, reuse, 1, 0.3)
+    _close(out, _sdpa(q, k, v, 0.3), TOL, "reuse of unchanged inputs vs sdpa")
+    assert np.array_equal(hit, (reuse == 0).astype(np.uint8))
+    assert np.array_equal(age, (reuse == 0).astype(np.int32))
+
+
+def pin_step_reuse_mixed(o):
+    """Q fixed, K/V move between steps: a reused pair must see the step-0 K/V
+    of its partition and a fresh pair the step-1 K/V, so each query partition
+    equals full attention over K/V stitched per partition (computed by sdpa)."""
+    r = _rng(12)
+    B, H, S, d, P = 1, 2, 40, 8, 5
+    n = S // P
+    q = r.normal(size=(B, H, S, d))
+    k0, v0 = r.normal(size=(B, H, S, d)), r.normal(size=(B, H, S, d))
+    k1, v1 = k0 + r.normal(size=k0.shape), v0 + r.normal(size=v0.shape)
+    anchor, reuse = _window_plans(P, 1)
+    reuse[0, 4] = o_STORE  # a forced-fresh far pair
+    cache = o.StateCache(P)
+    rows = np.array([0, 3, 9, 17, 22, 31, 38])
+    o.step(cache, q, k0, v0, anchor, 0, 0.4, rows=rows)
+    out, _, _, _ = o.step(cache, q, k1, v1, reuse, 1, 0.4, rows=rows)
+    for idx, row in enumerate(rows):
+        i = row // n
+        km, vm = k0.copy(), v0.copy()
+        for j in range(P):
+            if reuse[i, j] != o_REUSE:
+                km[..., j * n:(j + 1) * n, :] = k1[..., j * n:(j + 1) * n, :]
+                vm[..., j * n:(j + 1) * n, :] = v1[..., j * n:(j + 1) * n, :]
+        ref = _sdpa(q[..., row:row + 1, :], km, vm, 0.4)[..., 0, :]
+        _close(out[:, :, idx, :], ref, TOL, f"mixed row {row}")
+    assert cache.t_c[0, 4] == 1 and cache.t_c[0, 3] == 0
+
+
+PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_forms,
+        pin_compose_closed, pin_assoc_comm, pin_split_invariance, pin_single_partition,
+        pin_plan_golden, pin_step_all_fresh, pin_step_reuse_identical, pin_step_reuse_mixed]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_oracle_passes_pin(pin):
+    pin(as_oracle)
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each must fail at least one pin
+# ---------------------------------------------------------------------------
+
+_orig = {name: getattr(as_oracle, name) for name in
+         ("attention_state", "compose", "compose_pair", "resolve_plan", "step", "partition_bounds")}
+
+
+def _m_no_normalise(q, k, v, scale):
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    if k.shape[-2] == 0:
+        return as_oracle.empty_state(q.shape[:-1], v.shape[-1])
+    s = scale * (q @ np.swapaxes(k, -1, -2))
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=-1, keepdims=True)
+    return e @ v, (m + np.log(l))[..., 0]
+
+
+def _m_lse_unscaled(q, k, v, scale):
+    out, _ = _orig["attention_state"](q, k, v, scale)
+    _, lse = _orig["attention_state"](q, k, v, 1.0)
+    return out, lse
+
+
+def _m_transposed(q, k, v, scale):
+    return _orig["attention_state"](q, k, k, scale)
+
+
+def _m_log2(q, k, v, scale):
+    out, lse = _orig["attention_state"](q, k, v, scale)
+    return out, lse / math.log(2)
+
+
+def _m_compose_unnormalised(states):
+    states = list(states)
+    _, lse = _orig["compose"](states)
+    m = np.max(np.stack([l for _, l in states]), axis=0)
+    out = sum(np.exp(l - m)[..., None] * oo for oo, l in states)
+    return out, lse
+
+
+def _m_compose_sign(states):
+    states = [(oo, -l) for oo, l in states]
+    out, lse = _orig["compose"](states)
+    return out, -lse
+
+
+def _m_compose_drop_last(states):
+    states = list(states)
+    return _orig["compose"](states[:-1] if len(states) > 1 else states)
+
+
+def _m_pair_max_only(a, b):
+    out, _ = _orig["compose_pair"](a, b)
+    return out, np.maximum(a[1], b[1])
+
+
+def _m_age_sign(plan, t_c, t):
+    hit, age = _orig["resolve_plan"](plan, t_c, t)
+    return hit, -age
+
+
+def _m_hit_fresh(plan, t_c, t):
+    hit, age = _orig["resolve_plan"](plan, t_c, t)
+    return (1 - hit).astype(np.uint8), age
+
+
+def _m_store_all_fresh(cache, q, k, v, plan, t, scale, rows=None):
+    res = _orig["step"](cache, q, k, v, plan, t, scale, rows)
+    cache.t_c[np.asarray(plan) == 1] = t
+    return res
+
+
+def _m_bounds_shift(S, P):
+    b = _orig["partition_bounds"](S, P)
+    return b[1:] + b[:1]
+
+
+MUTANTS = {
+    "attention_state: OUT not normalised": ("attention_state", _m_no_normalise),
+    "attention_state: LSE without the scale": ("attention_state", _m_lse_unscaled),
+    "attention_state: K in place of V": ("attention_state", _m_transposed),
+    "attention_state: log2 instead of ln": ("attention_state", _m_log2),
+    "compose: weights not normalised": ("compose", _m_compose_unnormalised),
+    "compose: sign of the LSE": ("compose", _m_compose_sign),
+    "compose: drops a state": ("compose", _m_compose_drop_last),
+    "compose_pair: LSE = max": ("compose_pair", _m_pair_max_only),
+    "resolve_plan: age sign": ("resolve_plan", _m_age_sign),
+    "resolve_plan: hit on fresh": ("resolve_plan", _m_hit_fresh),
+    "step: stores plain-fresh pairs": ("step", _m_store_all_fresh),
+    "partition_bounds: off by one partition": ("partition_bounds", _m_bounds_shift),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(as_oracle, attr, fn)
+    failed = []
+    for pin in PINS:
+        try:
+            pin(as_oracle)
+        except Exception as e:  # noqa: BLE001 - any failure counts
+            failed.append(pin.__name__)
+    assert failed, f"no pin notices the planted mistake: {name}"
