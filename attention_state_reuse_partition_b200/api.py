@@ -1,0 +1,180 @@
+"""Python binding of the C ABI (include/as_partition.h), same names as the C
+entry points.  Argument marshalling only: tensors are passed by device
+pointer, outputs are allocated with torch when not given, streams are torch
+streams.  Every computation runs in the library's CUDA kernels."""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import (AS_BF16, AS_F32, AS_PLAN_FRESH, AS_PLAN_FRESH_STORE, AS_PLAN_REUSE, AsCacheStruct,
+                   AsError, LIB, check)
+
+__all__ = ["as_partition_attn", "as_compose", "as_cache_bytes", "as_cache_init", "as_plan_resolve", "as_step",
+           "as_device_status", "as_debug_timeout_probe", "as_version", "AsCache", "AsError",
+           "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE"]
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return AS_BF16
+    if t.dtype == torch.float32:
+        return AS_F32
+    raise AsError(_lib.AS_ERR_INVALID_ARG, f"unsupported input dtype {t.dtype}")
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda or not t.is_contiguous():
+        raise AsError(_lib.AS_ERR_INVALID_ARG, f"{name} must be a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def as_version() -> str:
+    return LIB.as_version().decode()
+
+
+def as_partition_attn(q, k, v, P: int, q_part: int, kv_parts: Sequence[int], compose: bool = True,
+                      scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """States of query partition ``q_part`` (or all rows, q_part=-1) against
+    the listed KV partitions; composed (compose=True) or one per partition."""
+    B, H, S, d = q.shape
+    R = S if q_part < 0 else S // P
+    scale = 1.0 / d ** 0.5 if scale is None else scale
+    planes = () if compose else (len(kv_parts),)
+    if out is None:
+        out = torch.empty(planes + (B, H, R, d), device=q.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty(planes + (B, H, R), device=q.device, dtype=torch.float32)
+    parts = (ctypes.c_int32 * len(kv_parts))(*[int(x) for x in kv_parts])
+    check(LIB.as_partition_attn(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q), B, H, S, d, P,
+                                float(scale), int(q_part), parts, len(kv_parts), 1 if compose else 0,
+                                _dev(out, "out"), _dev(lse, "lse"), _stream_ptr(stream)))
+    return out, lse
+
+
+def as_compose(outs, lses, out=None, lse=None, stream=None):
+    """Compose N states per row: outs [N, ..., d], lses [N, ...] (fp32)."""
+    N = outs.shape[0]
+    d = outs.shape[-1]
+    rows = lses[0].numel()
+    if out is None:
+        out = torch.empty(outs.shape[1:], device=outs.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty(lses.shape[1:], device=lses.device, dtype=torch.float32)
+    check(LIB.as_compose(_dev(outs, "outs"), _dev(lses, "lses"), N, rows, d, rows * d, rows,
+                         _dev(out, "out"), _dev(lse, "lse"), _stream_ptr(stream)))
+    return out, lse
+
+
+def as_cache_bytes(B: int, H: int, S: int, d: int, P: int) -> int:
+    return int(LIB.as_cache_bytes(B, H, S, d, P, AS_F32))
+
+
+class AsCache:
+    """A state cache: the C struct plus its device buffer (allocated with torch)."""
+
+    def __init__(self, B: int, H: int, S: int, d: int, P: int, device="cuda", buffer: Optional[torch.Tensor] = None):
+        nbytes = as_cache_bytes(B, H, S, d, P)
+        if nbytes == 0:
+            raise AsError(_lib.AS_ERR_INVALID_ARG, "invalid cache sizes")
+        if buffer is None:
+            buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.buffer = buffer
+        self.struct = AsCacheStruct()
+        check(LIB.as_cache_init(ctypes.byref(self.struct), buffer.data_ptr(), buffer.numel(), B, H, S, d, P, AS_F32))
+        self.B, self.H, self.S, self.d, self.P = B, H, S, d, P
+
+    @classmethod
+    def host_only(cls, B: int, H: int, S: int, d: int, P: int) -> "AsCache":
+        """A cache struct for host-side plan bookkeeping (as_plan_resolve) on a
+        machine without a GPU.  Its planes point at a placeholder address that
+        is never dereferenced; it must not be passed to as_step."""
+        self = cls.__new__(cls)
+        self.buffer = None
+        self.struct = AsCacheStruct()
+        check(LIB.as_cache_init(ctypes.byref(self.struct), 1 << 30, as_cache_bytes(B, H, S, d, P),
+                                B, H, S, d, P, AS_F32))
+        self.B, self.H, self.S, self.d, self.P = B, H, S, d, P
+        return self
+
+    def set_t_c(self, t_c) -> None:
+        """Overwrite the host-side store timestamps (for replaying bookkeeping)."""
+        flat = np.asarray(t_c, dtype=np.int32).reshape(-1)
+        for x in range(self.P * self.P):
+            self.struct.t_c[x] = int(flat[x])
+
+    @property
+    def t_c(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.struct.t_c)[: self.P * self.P].reshape(self.P, self.P).copy()
+
+    def planes(self):
+        """Views of the cache planes: OUT [P,B,H,S,d], LSE [P,B,H,S] (fp32)."""
+        n_out = self.P * self.B * self.H * self.S * self.d
+        n_lse = self.P * self.B * self.H * self.S
+        f = self.buffer.view(torch.float32)
+        return (f[:n_out].view(self.P, self.B, self.H, self.S, self.d),
+                f[n_out:n_out + n_lse].view(self.P, self.B, self.H, self.S))
+
+
+def as_cache_init(B, H, S, d, P, device="cuda", buffer=None) -> AsCache:
+    return AsCache(B, H, S, d, P, device=device, buffer=buffer)
+
+
+def _plan_bytes(plan, P):
+    arr = np.ascontiguousarray(np.asarray(plan, dtype=np.uint8).reshape(P * P))
+    return arr
+
+
+def as_plan_resolve(cache: AsCache, plan, step: int):
+    """Host-only plan check: returns (hit, age) as [P,P] numpy arrays."""
+    P = cache.P
+    arr = _plan_bytes(plan, P)
+    hit = np.zeros(P * P, dtype=np.uint8)
+    age = np.zeros(P * P, dtype=np.int32)
+    check(LIB.as_plan_resolve(ctypes.byref(cache.struct), arr.ctypes.data, int(step), hit.ctypes.data,
+                              age.ctypes.data))
+    return hit.reshape(P, P), age.reshape(P, P)
+
+
+def as_step(cache: AsCache, q, k, v, plan, step: int, scale: Optional[float] = None, out=None, lse=None,
+            stream=None):
+    """One step under a compute/reuse plan; returns (out, lse, hit, age)."""
+    B, H, S, d = q.shape
+    P = cache.P
+    scale = 1.0 / d ** 0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, S, d), device=q.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    arr = _plan_bytes(plan, P)
+    hit = np.zeros(P * P, dtype=np.uint8)
+    age = np.zeros(P * P, dtype=np.int32)
+    check(LIB.as_step(ctypes.byref(cache.struct), _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q),
+                      float(scale), arr.ctypes.data, int(step), _dev(out, "out"), _dev(lse, "lse"),
+                      hit.ctypes.data, age.ctypes.data, _stream_ptr(stream)))
+    return out, lse, hit.reshape(P, P), age.reshape(P, P)
+
+
+def as_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error bits;
+    raises AsError(AS_ERR_TIMEOUT) when a bounded wait ran out."""
+    bits = ctypes.c_uint32(0)
+    status = LIB.as_device_status(_stream_ptr(stream), ctypes.byref(bits))
+    if status not in (_lib.AS_OK, _lib.AS_ERR_TIMEOUT):
+        check(status)
+    if status == _lib.AS_ERR_TIMEOUT:
+        raise AsError(status, LIB.as_last_error().decode())
+    return bits.value
+
+
+def as_debug_timeout_probe(poll_budget: int = 64, stream=None) -> None:
+    check(LIB.as_debug_timeout_probe(int(poll_budget), _stream_ptr(stream)))

@@ -1,0 +1,331 @@
+// C-ABI boundary: argument checks, plan resolution, cache bookkeeping and
+// kernel dispatch.  Every step of the computation runs in the kernels; this
+// file only decides what to launch.
+//
+// Semantics follow DiTango (arXiv 2607.15650; review page: "What carries the
+// argument" for the attention state, Axiom & Free-Parameter Ledger Eq. 1-2 for
+// composition, Core claim and Referee Report "Summary" for fresh/reuse steps).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "as_kernels.h"
+#include "as_partition.h"
+
+namespace {
+
+constexpr uint32_t CACHE_MAGIC = 0x41535043u;  // "ASPC"
+thread_local std::string g_err;
+
+as_status fail(as_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+as_status ok() {
+  g_err.clear();
+  return AS_OK;
+}
+
+as_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(AS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+as_status check_shape(int B, int H, int S, int d, int P) {
+  if (B < 1 || H < 1 || S < 1) return fail(AS_ERR_INVALID_ARG, "B, H, S must be >= 1 (got %d, %d, %d)", B, H, S);
+  if (d != 64 && d != 128) return fail(AS_ERR_INVALID_ARG, "d must be 64 or 128 (got %d)", d);
+  if (P < 1 || P > AS_MAX_P) return fail(AS_ERR_INVALID_ARG, "P must be in [1, %d] (got %d)", AS_MAX_P, P);
+  if (S % P != 0) return fail(AS_ERR_INVALID_ARG, "S (%d) must be a multiple of P (%d)", S, P);
+  if (static_cast<long long>(B) * H > 65535) return fail(AS_ERR_INVALID_ARG, "B*H must be <= 65535");
+  if (static_cast<long long>(S) * d >= (1ll << 31)) return fail(AS_ERR_INVALID_ARG, "S*d too large");
+  return AS_OK;
+}
+
+// The kernels are built for sm_100a only.
+as_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(AS_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
+  return AS_OK;
+}
+
+as_status launch_attn(const asp::AttnLaunch& L, as_dtype dt, cudaStream_t st) {
+  cudaError_t e = (dt == AS_BF16) ? asp::launch_attn_tc_bf16(L, st) : asp::launch_attn_simt_f32(L, st);
+  if (e != cudaSuccess) return cuda_fail(e, dt == AS_BF16 ? "attention (tensor-core) launch" : "attention (fp32) launch");
+  return AS_OK;
+}
+
+void base_launch(asp::AttnLaunch& L, const void* q, const void* k, const void* v, int B, int H, int S, int d,
+                 int P, float scale) {
+  std::memset(&L, 0, sizeof(L));
+  L.q = q;
+  L.k = k;
+  L.v = v;
+  L.B = B;
+  L.H = H;
+  L.S = S;
+  L.d = d;
+  L.P = P;
+  L.n = S / P;
+  L.scale = scale;
+  L.poll_budget = 1u << 24;
+}
+
+// hit / age of a plan against cache timestamps; codes checked first, then misses
+as_status resolve(const as_cache* c, const uint8_t* plan, int step, uint8_t* hit, int32_t* age) {
+  const int P = c->P;
+  for (int x = 0; x < P * P; ++x)
+    if (plan[x] > AS_PLAN_FRESH_STORE)
+      return fail(AS_ERR_INVALID_ARG, "plan[%d][%d] = %d is not 0, 1 or 2", x / P, x % P, plan[x]);
+  for (int x = 0; x < P * P; ++x) {
+    if (plan[x] == AS_PLAN_REUSE && c->t_c[x] < 0)
+      return fail(AS_ERR_CACHE_MISS, "pair (%d, %d) is reused but its cache entry was never stored", x / P, x % P);
+  }
+  for (int x = 0; x < P * P; ++x) {
+    const bool r = plan[x] == AS_PLAN_REUSE;
+    if (hit) hit[x] = r ? 1 : 0;
+    if (age) age[x] = r ? step - c->t_c[x] : 0;
+  }
+  return AS_OK;
+}
+
+as_status check_cache(const as_cache* c) {
+  if (!c || c->magic != CACHE_MAGIC) return fail(AS_ERR_INVALID_ARG, "cache not initialised by as_cache_init");
+  return AS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* as_last_error(void) { return g_err.c_str(); }
+
+const char* as_version(void) { return "attention-state-reuse-partition b200 0.1 (sm_100a)"; }
+
+as_status as_partition_attn(const void* q, const void* k, const void* v, as_dtype dt, int B, int H, int S, int d,
+                            int P, float scale, int q_part, const int32_t* h_kv_parts, int n_kv_parts, int compose,
+                            float* out, float* lse, void* stream) {
+  as_status s = check_shape(B, H, S, d, P);
+  if (s != AS_OK) return s;
+  if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+  if (!q || !k || !v || !out || !lse) return fail(AS_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(AS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (q_part < -1 || q_part >= P) return fail(AS_ERR_INVALID_ARG, "q_part %d out of [-1, %d)", q_part, P);
+  if (!h_kv_parts || n_kv_parts < 1 || n_kv_parts > P)
+    return fail(AS_ERR_INVALID_ARG, "need 1..P KV partitions (got %d)", n_kv_parts);
+  if (compose != 0 && compose != 1) return fail(AS_ERR_INVALID_ARG, "compose must be 0 or 1");
+  if (!(scale > 0.f)) return fail(AS_ERR_INVALID_ARG, "scale must be > 0");
+  asp::AttnLaunch L;
+  base_launch(L, q, k, v, B, H, S, d, P, scale);
+  const int R = q_part >= 0 ? S / P : S;
+  L.n_blocks = 1;
+  L.block_rows = R;
+  L.block_row0 = q_part >= 0 ? q_part * (S / P) : 0;
+  for (int x = 0; x < n_kv_parts; ++x) {
+    const int j = h_kv_parts[x];
+    if (j < 0 || j >= P) return fail(AS_ERR_INVALID_ARG, "KV partition %d out of [0, %d)", j, P);
+    if (L.code[j] != AS_KCODE_SKIP) return fail(AS_ERR_INVALID_ARG, "KV partition %d listed twice", j);
+    L.code[j] = compose ? AS_KCODE_COMPOSE : AS_KCODE_EMIT;
+    L.dest_of[j] = static_cast<int8_t>(x);
+  }
+  L.out = out;
+  L.lse = lse;
+  L.out_rows = R;
+  L.out_row0 = L.block_row0;
+  L.dst_out = out;
+  L.dst_lse = lse;
+  L.dst_rows = R;
+  L.dst_row0 = L.block_row0;
+  L.dst_plane_out = static_cast<long long>(B) * H * R * d;
+  L.dst_plane_lse = static_cast<long long>(B) * H * R;
+  if ((s = check_device()) != AS_OK) return s;
+  if ((s = launch_attn(L, dt, static_cast<cudaStream_t>(stream))) != AS_OK) return s;
+  return ok();
+}
+
+as_status as_compose(const float* outs, const float* lses, int n_states, int64_t rows, int d,
+                     int64_t state_stride_out, int64_t state_stride_lse, float* out, float* lse, void* stream) {
+  if (d != 64 && d != 128) return fail(AS_ERR_INVALID_ARG, "d must be 64 or 128 (got %d)", d);
+  if (n_states < 1) return fail(AS_ERR_INVALID_ARG, "n_states must be >= 1");
+  if (rows < 0) return fail(AS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (rows == 0) return ok();
+  if (!outs || !lses || !out || !lse) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(outs) || !aligned16(out)) return fail(AS_ERR_INVALID_ARG, "OUT pointers must be 16-byte aligned");
+  if (n_states > 1 && (state_stride_out < rows * d || state_stride_lse < rows || (state_stride_out % 4) != 0))
+    return fail(AS_ERR_INVALID_ARG, "state strides must cover a whole state (and OUT stride be a multiple of 4)");
+  asp::ComposeStrided a;
+  a.outs = outs;
+  a.lses = lses;
+  a.n_states = n_states;
+  a.d = d;
+  a.rows = rows;
+  a.stride_out = state_stride_out;
+  a.stride_lse = state_stride_lse;
+  a.out = out;
+  a.lse = lse;
+  as_status s = check_device();
+  if (s != AS_OK) return s;
+  cudaError_t e = asp::launch_compose_strided(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "compose launch");
+  return ok();
+}
+
+size_t as_cache_bytes(int B, int H, int S, int d, int P, as_dtype cache_dt) {
+  if (cache_dt != AS_F32) return 0;
+  if (check_shape(B, H, S, d, P) != AS_OK) return 0;
+  return static_cast<size_t>(P) * B * H * S * (d + 1) * sizeof(float);
+}
+
+as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, as_dtype cache_dt) {
+  if (!c) return fail(AS_ERR_INVALID_ARG, "null cache struct");
+  if (cache_dt != AS_F32) return fail(AS_ERR_UNSUPPORTED, "only fp32 cache entries are built");
+  as_status s = check_shape(B, H, S, d, P);
+  if (s != AS_OK) return s;
+  const size_t need = as_cache_bytes(B, H, S, d, P, cache_dt);
+  if (!buf || (reinterpret_cast<uintptr_t>(buf) & 255u) != 0)
+    return fail(AS_ERR_INVALID_ARG, "cache buffer must be non-null and 256-byte aligned");
+  if (bytes < need) return fail(AS_ERR_INVALID_ARG, "cache buffer has %zu bytes, needs %zu", bytes, need);
+  std::memset(c, 0, sizeof(*c));
+  c->magic = CACHE_MAGIC;
+  c->B = B;
+  c->H = H;
+  c->S = S;
+  c->d = d;
+  c->P = P;
+  c->cache_dt = cache_dt;
+  c->out_planes = static_cast<float*>(buf);
+  c->lse_planes = c->out_planes + static_cast<size_t>(P) * B * H * S * d;
+  for (int x = 0; x < AS_MAX_P * AS_MAX_P; ++x) c->t_c[x] = -1;
+  return ok();
+}
+
+as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step, uint8_t* h_hit, int32_t* h_age) {
+  as_status s = check_cache(c);
+  if (s != AS_OK) return s;
+  if (!h_plan) return fail(AS_ERR_INVALID_ARG, "null plan");
+  if ((s = resolve(c, h_plan, step, h_hit, h_age)) != AS_OK) return s;
+  return ok();
+}
+
+as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
+                  const uint8_t* h_plan, int step, float* out, float* lse, uint8_t* h_hit, int32_t* h_age,
+                  void* stream) {
+  as_status s = check_cache(c);
+  if (s != AS_OK) return s;
+  if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+  if (!q || !k || !v || !out || !lse || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(AS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (!(scale > 0.f)) return fail(AS_ERR_INVALID_ARG, "scale must be > 0");
+  const int B = c->B, H = c->H, S = c->S, d = c->d, P = c->P, n = S / P;
+  uint8_t hit[AS_MAX_P * AS_MAX_P];
+  int32_t age[AS_MAX_P * AS_MAX_P];
+  if ((s = resolve(c, h_plan, step, hit, age)) != AS_OK) return s;
+  if ((s = check_device()) != AS_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // fresh pairs: composite of the plain-fresh partitions -> out/lse, stored
+  // pairs -> their cache planes
+  asp::AttnLaunch L;
+  base_launch(L, q, k, v, B, H, S, d, P, scale);
+  L.n_blocks = P;
+  L.block_rows = n;
+  L.block_row0 = 0;
+  bool any_fresh = false, need_compose = false;
+  for (int i = 0; i < P; ++i) {
+    for (int j = 0; j < P; ++j) {
+      const uint8_t pc = h_plan[i * P + j];
+      L.code[i * P + j] = pc == AS_PLAN_FRESH ? AS_KCODE_COMPOSE : pc == AS_PLAN_FRESH_STORE ? AS_KCODE_EMIT
+                                                                                            : AS_KCODE_SKIP;
+      any_fresh |= pc != AS_PLAN_REUSE;
+      need_compose |= pc != AS_PLAN_FRESH;
+    }
+  }
+  for (int j = 0; j < P; ++j) L.dest_of[j] = static_cast<int8_t>(j);
+  L.out = out;
+  L.lse = lse;
+  L.out_rows = S;
+  L.out_row0 = 0;
+  L.dst_out = c->out_planes;
+  L.dst_lse = c->lse_planes;
+  L.dst_rows = S;
+  L.dst_row0 = 0;
+  L.dst_plane_out = static_cast<long long>(B) * H * S * d;
+  L.dst_plane_lse = static_cast<long long>(B) * H * S;
+  if (any_fresh && (s = launch_attn(L, dt, st)) != AS_OK) return s;
+
+  // final composition: composite + stored fresh states + reused entries
+  if (need_compose) {
+    asp::ComposePlan a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = B;
+    a.H = H;
+    a.S = S;
+    a.d = d;
+    a.P = P;
+    a.n = n;
+    for (int i = 0; i < P; ++i) {
+      int cnt = 0;
+      bool has_fresh = false, has_other = false;
+      for (int j = 0; j < P; ++j) {
+        has_fresh |= h_plan[i * P + j] == AS_PLAN_FRESH;
+        has_other |= h_plan[i * P + j] != AS_PLAN_FRESH;
+      }
+      if (!has_other) {
+        a.nsrc[i] = 0;  // the composite already is the final state
+        continue;
+      }
+      if (has_fresh) a.src[i][cnt++] = -1;
+      for (int j = 0; j < P; ++j)
+        if (h_plan[i * P + j] != AS_PLAN_FRESH) a.src[i][cnt++] = static_cast<int8_t>(j);
+      a.nsrc[i] = static_cast<uint8_t>(cnt);
+    }
+    a.cache_out = c->out_planes;
+    a.cache_lse = c->lse_planes;
+    a.plane_out = L.dst_plane_out;
+    a.plane_lse = L.dst_plane_lse;
+    a.out = out;
+    a.lse = lse;
+    cudaError_t e = asp::launch_compose_plan(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "step compose launch");
+  }
+
+  for (int x = 0; x < P * P; ++x)
+    if (h_plan[x] == AS_PLAN_FRESH_STORE) c->t_c[x] = step;
+  if (h_hit) std::memcpy(h_hit, hit, static_cast<size_t>(P) * P);
+  if (h_age) std::memcpy(h_age, age, static_cast<size_t>(P) * P * sizeof(int32_t));
+  return ok();
+}
+
+as_status as_device_status(void* stream, uint32_t* h_bits) {
+  unsigned int bits = 0;
+  cudaError_t e = asp::read_and_clear_dev_error(&bits, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "device status");
+  if (h_bits) *h_bits = bits;
+  if (bits & AS_DEVERR_TIMEOUT) return fail(AS_ERR_TIMEOUT, "a kernel's bounded wait ran out (bits 0x%x)", bits);
+  return ok();
+}
+
+as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream) {
+  as_status s = check_device();
+  if (s != AS_OK) return s;
+  cudaError_t e = asp::launch_timeout_probe(poll_budget, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "timeout probe launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Internal interface between the C-ABI dispatcher (as_api.cu) and the kernels.
+// Not installed; the public boundary is include/as_partition.h.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#ifndef AS_MAX_P
+#define AS_MAX_P 64
+#endif
+
+// kernel codes for one (query row block, KV partition) pair
+#define AS_KCODE_SKIP 0     // partition not read
+#define AS_KCODE_COMPOSE 1  // partition folded into the block's composite state
+#define AS_KCODE_EMIT 2     // partition emitted as its own state to a destination plane
+
+// bits of the device error word
+#define AS_DEVERR_TIMEOUT 1u
+
+namespace asp {
+
+// Everything an attention launch needs, passed by value as a kernel parameter.
+struct AttnLaunch {
+  const void* q;  // [B,H,S,d] (used by the SIMT path; the TMA path reads via tensor maps)
+  const void* k;
+  const void* v;
+  int B, H, S, d, P, n;  // n = S / P
+  float scale;
+  // query rows: n_blocks blocks of block_rows rows starting at block_row0; block b
+  // uses row b of `code` ([n_blocks][P])
+  int n_blocks, block_rows, block_row0;
+  uint8_t code[AS_MAX_P * AS_MAX_P];
+  int8_t dest_of[AS_MAX_P];  // destination plane of each AS_KCODE_EMIT partition
+  // composite output: row s of head bh at ((bh * out_rows) + s - out_row0)
+  float* out;
+  float* lse;
+  int out_rows, out_row0;
+  // emitted planes: plane p, row s of head bh at p * plane + (bh * dst_rows + s - dst_row0)
+  float* dst_out;
+  float* dst_lse;
+  int dst_rows, dst_row0;
+  long long dst_plane_out, dst_plane_lse;
+  unsigned int poll_budget;
+};
+
+// compose of N states per row with strided state storage (as_compose)
+struct ComposeStrided {
+  const float* outs;
+  const float* lses;
+  int n_states, d;
+  long long rows;
+  long long stride_out, stride_lse;  // distance between consecutive states, in elements
+  float* out;
+  float* lse;
+};
+
+// final compose of a step: composite (in out/lse) + cache planes, chosen per
+// query partition from the step plan
+struct ComposePlan {
+  int B, H, S, d, P, n;
+  int8_t src[AS_MAX_P][AS_MAX_P + 1];  // per query partition: -1 = composite, j = cache plane j
+  uint8_t nsrc[AS_MAX_P];
+  const float* cache_out;
+  const float* cache_lse;
+  long long plane_out, plane_lse;
+  float* out;  // [B,H,S,d]: holds the composite on entry (where used), the final state on exit
+  float* lse;
+};
+
+cudaError_t launch_attn_tc_bf16(const AttnLaunch& L, cudaStream_t st);
+cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st);
+cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st);
+cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st);
+cudaError_t launch_timeout_probe(unsigned int poll_budget, cudaStream_t st);
+cudaError_t read_and_clear_dev_error(unsigned int* bits, cudaStream_t st);
+
+}  // namespace asp

@@ -1,0 +1,216 @@
+// State composition kernels (HBM-bound).
+//
+// DiTango (arXiv 2607.15650; review page, Axiom & Free-Parameter Ledger,
+// Eq. 1-2): attention states compose associatively and commutatively.  For N
+// states of one query row, LSE = m + ln sum_k exp(LSE_k - m) with m = max_k
+// LSE_k, and OUT = sum_k exp(LSE_k - LSE) * OUT_k.  A row whose states are all
+// empty (LSE = -inf) stays empty: OUT = 0, LSE = -inf.
+//
+// One warp composes a block of up to 8 consecutive rows that share their
+// source list.  Lane k holds the LSEs of source k for the 8 rows (one 32-byte
+// sector per source), so the max and the sum are warp reductions; the OUT
+// rows are read with 128-bit loads, one 512-byte row per warp instruction
+// (d = 128), several sources in flight per lane.  Every input byte is read
+// once from HBM (the LSE re-reads of the third pass hit L1) and the output is
+// written once.  Grids are persistent: 148 SMs x 8 CTAs x 8 warps.
+#include "as_device.cuh"
+
+namespace asp {
+namespace {
+
+constexpr int RB = 8;        // rows per warp block
+constexpr int WARPS = 8;     // warps per CTA
+constexpr int SM_COUNT = 148;
+
+template <int D>
+struct Vec;
+template <>
+struct Vec<128> {
+  using T = float4;
+  static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  static __device__ __forceinline__ void fma(float4& a, float c, const float4& x) {
+    a.x = fmaf(c, x.x, a.x);
+    a.y = fmaf(c, x.y, a.y);
+    a.z = fmaf(c, x.z, a.z);
+    a.w = fmaf(c, x.w, a.w);
+  }
+};
+template <>
+struct Vec<64> {
+  using T = float2;
+  static __device__ __forceinline__ float2 zero() { return make_float2(0.f, 0.f); }
+  static __device__ __forceinline__ void fma(float2& a, float c, const float2& x) {
+    a.x = fmaf(c, x.x, a.x);
+    a.y = fmaf(c, x.y, a.y);
+  }
+};
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Composes rows [row0, row0+nr) (nr <= RB) of `nsrc` sources.  src(k) gives the
+// base pointers (out_base, lse_base) of source k such that row r's state is at
+// out_base + r*D and lse_base + r.  The output may alias a source: every source
+// row is read before the output row is written, by the same warp.
+template <int D, class SrcFn>
+__device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, SrcFn src, float* out,
+                                             float* lse, int lane) {
+  using V = Vec<D>;
+  using T = typename V::T;
+  float m[RB], tot[RB];
+#pragma unroll
+  for (int rr = 0; rr < RB; ++rr) m[rr] = -INFINITY;
+  for (int k0 = 0; k0 < nsrc; k0 += 32) {
+    const int k = k0 + lane;
+    if (k < nsrc) {
+      const float* lb = src(k).second + row0;
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr)
+        if (rr < nr) m[rr] = fmaxf(m[rr], lb[rr]);
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < RB; ++rr) {
+    m[rr] = warp_max(m[rr]);
+    tot[rr] = 0.f;
+  }
+  for (int k0 = 0; k0 < nsrc; k0 += 32) {
+    const int k = k0 + lane;
+    if (k < nsrc) {
+      const float* lb = src(k).second + row0;
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr)
+        if (rr < nr && m[rr] != -INFINITY) tot[rr] += expf(lb[rr] - m[rr]);
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < RB; ++rr) tot[rr] = warp_sum(tot[rr]);
+
+  T acc[RB];
+#pragma unroll
+  for (int rr = 0; rr < RB; ++rr) acc[rr] = V::zero();
+  for (int k0 = 0; k0 < nsrc; k0 += 32) {
+    const int k = k0 + lane;
+    float coef[RB];
+    if (k < nsrc) {
+      const float* lb = src(k).second + row0;
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr)
+        coef[rr] = (rr < nr && tot[rr] > 0.f) ? expf(lb[rr] - m[rr]) / tot[rr] : 0.f;
+    } else {
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr) coef[rr] = 0.f;
+    }
+    const int kn = min(32, nsrc - k0);
+#pragma unroll
+    for (int rr = 0; rr < RB; ++rr) {
+      if (rr >= nr) break;
+      int kk = 0;
+      for (; kk + 8 <= kn; kk += 8) {
+        T x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          x[u] = reinterpret_cast<const T*>(src(k0 + kk + u).first + (row0 + rr) * D)[lane];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk + u), x[u]);
+      }
+      for (; kk < kn; ++kk) {
+        const T x = reinterpret_cast<const T*>(src(k0 + kk).first + (row0 + rr) * D)[lane];
+        V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk), x);
+      }
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < RB; ++rr) {
+    if (rr >= nr) break;
+    reinterpret_cast<T*>(out + (row0 + rr) * D)[lane] = acc[rr];
+    if (lane == 0) lse[row0 + rr] = tot[rr] > 0.f ? m[rr] + logf(tot[rr]) : -INFINITY;
+  }
+}
+
+struct Ptrs {
+  const float* first;
+  const float* second;
+};
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32) compose_strided_kernel(const __grid_constant__ ComposeStrided a) {
+  const int lane = threadIdx.x & 31;
+  const long long nblk = (a.rows + RB - 1) / RB;
+  const long long gw = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
+  const long long stride = static_cast<long long>(gridDim.x) * WARPS;
+  auto src = [&](int k) {
+    return Ptrs{a.outs + k * a.stride_out, a.lses + k * a.stride_lse};
+  };
+  for (long long b = gw; b < nblk; b += stride) {
+    const long long row0 = b * RB;
+    const int nr = static_cast<int>(min(static_cast<long long>(RB), a.rows - row0));
+    compose_rows<D>(row0, nr, a.n_states, src, a.out, a.lse, lane);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32) compose_plan_kernel(const __grid_constant__ ComposePlan a) {
+  const int lane = threadIdx.x & 31;
+  const int bpp = (a.n + RB - 1) / RB;  // warp blocks per (head, partition)
+  const long long nblk = static_cast<long long>(a.B) * a.H * a.P * bpp;
+  const long long gw = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
+  const long long stride = static_cast<long long>(gridDim.x) * WARPS;
+  for (long long b = gw; b < nblk; b += stride) {
+    const int rb = static_cast<int>(b % bpp);
+    const int i = static_cast<int>((b / bpp) % a.P);
+    if (a.nsrc[i] == 0) continue;  // the composite already is the final state
+    const long long bh = b / (static_cast<long long>(bpp) * a.P);
+    const int s0 = i * a.n + rb * RB;
+    const int nr = min(RB, (i + 1) * a.n - s0);
+    const long long row0 = bh * a.S + s0;
+    const int8_t* list = a.src[i];
+    auto src = [&](int k) {
+      const int j = list[k];
+      if (j < 0) return Ptrs{a.out, a.lse};
+      return Ptrs{a.cache_out + j * a.plane_out, a.cache_lse + j * a.plane_lse};
+    };
+    compose_rows<D>(row0, nr, a.nsrc[i], src, a.out, a.lse, lane);
+  }
+}
+
+long long grid_for(long long nblk) {
+  const long long ctas = (nblk + WARPS - 1) / WARPS;
+  return ctas < SM_COUNT * 8 ? (ctas > 0 ? ctas : 1) : SM_COUNT * 8;
+}
+
+}  // namespace
+
+cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st) {
+  const long long nblk = (a.rows + RB - 1) / RB;
+  const unsigned grid = static_cast<unsigned>(grid_for(nblk));
+  if (a.d == 128)
+    compose_strided_kernel<128><<<grid, WARPS * 32, 0, st>>>(a);
+  else if (a.d == 64)
+    compose_strided_kernel<64><<<grid, WARPS * 32, 0, st>>>(a);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st) {
+  const long long nblk = static_cast<long long>(a.B) * a.H * a.P * ((a.n + RB - 1) / RB);
+  const unsigned grid = static_cast<unsigned>(grid_for(nblk));
+  if (a.d == 128)
+    compose_plan_kernel<128><<<grid, WARPS * 32, 0, st>>>(a);
+  else if (a.d == 64)
+    compose_plan_kernel<64><<<grid, WARPS * 32, 0, st>>>(a);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace asp

@@ -1,0 +1,408 @@
+"""Benchmark: fresh-partition attention TFLOP/s (and state-compose GB/s) on B200.
+
+One step = one ``as_step`` over the FLUX-like image-DiT attention workload
+(B=1, H=24, S=4608 = 4096 image + 512 text tokens, d=128, bf16 in / fp32
+states, P=8 partitions of 576, every pair fresh and composed): plan
+resolution, the partition states of all eight KV partitions and their
+composition, on the tensor cores.  FLOPs counted: 4*B*H*S*S*d per step (QK^T
+and PV, fresh pairs only).  Inputs are resident in HBM; the L2 is flushed
+(a 256 MiB write) before every timed step, outside the timed events.
+
+Also reported on the same line (same run):
+* ``e2e``: the same step through the public API from pinned HOST buffers,
+  with the host->device copy of Q, K, V and the device->host copy of OUT and
+  LSE inside the timed region;
+* ``roofline``: the attention kernel against the measured dense bf16 peak;
+* ``secondary``: the state-compose kernel on the compose-bound workload (GB/s
+  against measured HBM copy bandwidth) and the two-step video reuse workload
+  (fresh TFLOP/s, reuse-compose GB/s, reuse MSE against full attention);
+* ``cpu_baseline``: the float64 oracle on the host cores on a sample of rows.
+
+``--impl reference`` times the float64 oracle instead (the only reference
+implementation of this method available here), on the host cores, on samples
+of the same workload, and prints the same metric.
+
+Multi-GPU: every rank runs its own replica of the workload (the path shards
+by heads and batches with no exchange step); value = all ranks' FLOPs / the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_state_reuse_partition_b200 import workloads as W  # noqa: E402
+
+METRIC = "fresh-partition attn TFLOP/s & compose GB/s at 1 B200; % of bf16/HBM roofline"
+WORKLOAD = "flux_image"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def attn_flops(s) -> float:
+    return 4.0 * s.B * s.H * s.S * s.S * s.d
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] not in ("", "[N/A]"))}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of rows
+# ---------------------------------------------------------------------------
+
+def oracle_sample(s, q, k, v, rows_per_partition: int, heads):
+    """Times the oracle's all-fresh step on a seeded sample of query rows
+    (all keys, the given heads).  Returns (seconds, flops)."""
+    from oracle import as_oracle as O
+    rows = W.sample_rows(s, rows_per_partition).numpy()
+    qn = q[:, heads][:, :, rows].float().cpu().double().numpy()
+    kn = k[:, heads].float().cpu().double().numpy()
+    vn = v[:, heads].float().cpu().double().numpy()
+    cache = O.StateCache(s.P)
+    plan = np.ones((s.P, s.P), np.uint8)
+    # the oracle's step takes full-length Q and selects `rows`; pad Q
+    qfull = np.zeros((s.B, len(heads), s.S, s.d))
+    qfull[:, :, rows] = qn
+    t0 = time.perf_counter()
+    O.step(cache, qfull, kn, vn, plan, 0, s.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * s.B * len(heads) * len(rows) * s.S * s.d
+    return dt, flops
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info()), default=0)
+        if n:
+            return n
+    except Exception:  # noqa: BLE001
+        pass
+    return os.cpu_count()
+
+
+# ---------------------------------------------------------------------------
+# the timed legs
+# ---------------------------------------------------------------------------
+
+def run_own(args, rank, world, device):
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec(WORKLOAD)
+    q, k, v = W.flux_qkv(s, device=device)
+    plan = W.all_fresh_plan(s.P).numpy()
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    out = torch.empty((s.B, s.H, s.S, s.d), device=device, dtype=torch.float32)
+    lse = torch.empty((s.B, s.H, s.S), device=device, dtype=torch.float32)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=device, dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.as_step(cache, q, k, v, plan, 0, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))           # L2 flush, keeps the GPU busy across the launch gap
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(times) / len(times)
+    api.as_device_status()
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = t.item()
+    flops = attn_flops(s)
+    value = flops * world / (ms_max * 1e-3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        api.as_step(cache, dq, dk, dv, plan, 0, out=out, lse=lse)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = t.item()
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = hout.numel() * 4 + hlse.numel() * 4
+    assert torch.allclose(hout.to(device), out), "e2e output differs from the device-resident run"
+
+    result = {
+        "ms": ms, "ms_max": ms_max, "value": value, "flops": flops,
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clk.summary(), "gpu_launches": args.steps,
+        "step_ms": times,
+    }
+    del cache, flush
+    torch.cuda.empty_cache()
+    return result, (q, k, v, s)
+
+
+def run_compose(args, device):
+    """Compose-bound workload: 32 fp32 states per row merged into one."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec("compose_bound")
+    outs, lses = W.compose_states(s, device=device)
+    out = torch.empty(outs.shape[1:], device=device)
+    lse = torch.empty(lses.shape[1:], device=device)
+    for _ in range(3):
+        api.as_compose(outs, lses, out=out, lse=lse)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+    for a, b in ev:
+        a.record()
+        api.as_compose(outs, lses, out=out, lse=lse)
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    rows = outs.shape[1]
+    nbytes = (s.n_states + 1) * rows * (s.d + 1) * 4
+    del outs, lses, out, lse
+    torch.cuda.empty_cache()
+    return {"workload": "compose_bound", "ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms * 1e-3) / 1e9}
+
+
+def run_reuse(args, device):
+    """Two-step video reuse: anchor step then a reuse step (window 2)."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec("video_reuse")
+    steps = [(q, k, v) for _, q, k, v in W.video_trajectory(s, device=device)]
+    plans = [W.plan_for_step(s, t).numpy() for t in range(s.steps)]
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    out = torch.empty((s.B, s.H, s.S, s.d), device=device)
+    lse = torch.empty((s.B, s.H, s.S), device=device)
+    q1, k1, v1 = steps[1]
+    n_fresh = int((plans[1] != W.PLAN_REUSE).sum())
+    n_reuse = int((plans[1] == W.PLAN_REUSE).sum())
+    fresh_flops = 4.0 * s.B * s.H * n_fresh * s.n * s.n * s.d
+    times = []
+    for rep in range(4):
+        c = api.AsCache(s.B, s.H, s.S, s.d, s.P, buffer=cache.buffer)
+        api.as_step(c, *steps[0], plans[0], 0, out=out, lse=lse)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        api.as_step(c, q1, k1, v1, plans[1], 1, out=out, lse=lse)
+        b.record()
+        torch.cuda.synchronize()
+        if rep > 0:
+            times.append(a.elapsed_time(b))
+    ms = statistics.mean(times)
+    full_o, _ = api.as_partition_attn(q1, k1, v1, s.P, -1, list(range(s.P)))
+    torch.cuda.synchronize()
+    mse = torch.mean((out - full_o) ** 2).item()
+    state_bytes = s.B * s.H * s.n * (s.d + 1) * 4
+    reuse_bytes = n_reuse * state_bytes
+    del cache, steps, full_o
+    torch.cuda.empty_cache()
+    return {"workload": "video_reuse step t", "ms": ms, "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
+            "fresh_tflops_whole_step": fresh_flops / (ms * 1e-3) / 1e12, "reuse_bytes": reuse_bytes,
+            "reuse_mse_vs_full": mse}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["own", "reference"], default="own")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--cpu-sample-rows", type=int, default=48)
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    peaks = load_peaks()
+    res, (q, k, v, s) = run_own(args, rank, world, device)
+    secondary = {}
+    if not args.no_secondary and world == 1:
+        comp = run_compose(args, device)
+        comp["frac_of_hbm"] = comp["GB/s"] / peaks["hbm_gbs"]
+        secondary["compose"] = comp
+        secondary["reuse"] = run_reuse(args, device)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        heads = [0, 11, 23]
+        dt, fl = oracle_sample(s, q, k, v, args.cpu_sample_rows, heads)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"{args.cpu_sample_rows} query rows per partition x {len(heads)} heads of {WORKLOAD}, "
+                         f"all {s.S} keys, float64 ({dt:.1f} s)"}
+
+    ms = res["ms_max"]
+    achieved = res["flops"] / (res["ms"] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": round(res["value"], 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: B=1 H=24 S=4608 (4096 image + 512 text) d=128, P=8 partitions "
+                               f"of 576, all pairs fresh and composed", "global_batch": world, "seq_len": s.S,
+                   "parallelism": f"replicas{world}" if world > 1 else "single", "l2": "flushed (256 MiB write) "
+                   "before every timed step"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "attn_tc_kernel<128>", "peak_source": f"{peaks['source']} bf16 burst"},
+        "e2e": res["e2e"], "clocks": res["clocks"], "gpu_launches": res["gpu_launches"],
+    }
+    if cpu:
+        line["cpu_baseline"] = cpu
+    if secondary:
+        line["secondary"] = secondary
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
+def run_reference(args, rank, world):
+    """The float64 oracle on the host cores, each step a bounded sample of the
+    workload's query rows (all keys, three heads)."""
+    if rank != 0:
+        return
+    s = W.spec(WORKLOAD)
+    q, k, v = W.flux_qkv(s)
+    heads = [0, 11, 23]
+    rows = 8
+    for _ in range(args.warmup):
+        oracle_sample(s, q, k, v, rows, heads)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(s, q, k, v, rows, heads)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = f"{rows} query rows per partition x {len(heads)} heads of {WORKLOAD}, all {s.S} keys, float64"
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{WORKLOAD}: B=1 H=24 S=4608 d=128, P=8, all pairs fresh (sampled rows)",
+                   "global_batch": 1, "seq_len": s.S, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

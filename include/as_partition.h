@@ -1,0 +1,157 @@
+/* Attention states over sequence partitions, with cached-state reuse: C ABI.
+ *
+ * The operations follow DiTango ("DiTango: Cost-Effective Parallel Diffusion
+ * Generation with Selective Attention State Reuse", arXiv 2607.15650), as
+ * summarised on its pith.science review page:
+ *   - "What carries the argument": for a sequence (KV) partition j the
+ *     attention state is AS(j) = (OUT(j), LSE(j)), the partial attention
+ *     output of j's keys and the log-sum-exp of their scores;
+ *   - Axiom & Free-Parameter Ledger, Eq. 1-2: states compose associatively and
+ *     commutatively by LSE weighting;
+ *   - Core claim and Referee Report "Summary": at a denoising step, fresh
+ *     states are computed for some partitions and cached composed states from
+ *     earlier steps are reused for the others, under a per-(query partition,
+ *     KV partition) compute/reuse plan; anchor steps compute every state.
+ *
+ * Conventions for every call:
+ *   - Tensors are row-major.  Q, K, V are [B, H, S, d] (d contiguous); a state
+ *     is OUT [.., S, d] fp32 (normalised partial output) and LSE [.., S] fp32
+ *     (natural log, softmax scale included).  The empty state is OUT = 0,
+ *     LSE = -inf.
+ *   - Partition j covers tokens [j*n, (j+1)*n) with n = S / P.  Query
+ *     partitions use the same split.  Attention is bidirectional (no mask).
+ *   - Pointers without an h_ prefix are device pointers; h_ pointers are host
+ *     memory.  The caller owns all memory.  The library allocates no device
+ *     memory and does not synchronise the caller's stream; results follow
+ *     stream order on `stream` (a cudaStream_t, NULL = legacy default stream).
+ *   - Device pointers must be 16-byte aligned.  Supported: d in {64, 128},
+ *     1 <= P <= AS_MAX_P, S % P == 0, B*H <= 65535.
+ *   - Every call returns an as_status; on failure as_last_error() gives a
+ *     message (thread-local).  Argument errors are reported before any launch.
+ */
+#ifndef AS_PARTITION_H
+#define AS_PARTITION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define AS_MAX_P 64
+
+typedef enum {
+  AS_OK = 0,
+  AS_ERR_INVALID_ARG = 1,  /* shapes, alignment, plan values, cache mismatch */
+  AS_ERR_UNSUPPORTED = 2,  /* valid request outside the built paths */
+  AS_ERR_CACHE_MISS = 3,   /* the plan reuses a pair whose entry was never stored */
+  AS_ERR_CUDA = 4,         /* a CUDA runtime call failed (message in as_last_error) */
+  AS_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see as_device_status) */
+} as_status;
+
+typedef enum {
+  AS_F32 = 0,   /* fp32 inputs: CUDA-core path */
+  AS_BF16 = 1   /* bf16 inputs, fp32 accumulation and states: tensor-core path */
+} as_dtype;
+
+/* plan codes for as_step (uint8 per (query partition i, KV partition j)) */
+#define AS_PLAN_REUSE 0        /* read the cached state of (i, j) */
+#define AS_PLAN_FRESH 1        /* compute the state of (i, j); cache untouched */
+#define AS_PLAN_FRESH_STORE 2  /* compute the state of (i, j) and refresh its cache entry */
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* as_last_error(void);
+
+/* Library version string. */
+const char* as_version(void);
+
+/* Attention states of one query partition (or of all query rows) against a
+ * list of KV partitions.  DiTango review, "What carries the argument" (the
+ * state) and Eq. 1-2 (composition).
+ *
+ *   q, k, v       [B,H,S,d] of type dt.
+ *   scale         softmax scale (scores are scale * <q, k>).
+ *   q_part        query partition i in [0, P), or -1 for all S query rows.
+ *   h_kv_parts    host array of n_kv_parts distinct KV partition indices.
+ *   compose = 1:  one state per query row, the composition of the listed
+ *                 partitions' states: out [B,H,R,d], lse [B,H,R] with R = n
+ *                 (q_part >= 0) or S (q_part = -1).
+ *   compose = 0:  one state per listed partition: out [n_kv_parts,B,H,R,d],
+ *                 lse [n_kv_parts,B,H,R]; plane k holds h_kv_parts[k].
+ * Errors: AS_ERR_INVALID_ARG for a bad shape, index, duplicate or alignment;
+ * AS_ERR_CUDA if the launch fails. */
+as_status as_partition_attn(const void* q, const void* k, const void* v, as_dtype dt,
+                            int B, int H, int S, int d, int P, float scale,
+                            int q_part, const int32_t* h_kv_parts, int n_kv_parts, int compose,
+                            float* out, float* lse, void* stream);
+
+/* Compose n_states states per row into one (DiTango review, Eq. 1-2).
+ *   State k, row r: OUT at outs + k*state_stride_out + r*d, LSE at
+ *   lses + k*state_stride_lse + r (strides in elements).  rows >= 0.
+ *   out [rows, d], lse [rows].  out/lse must not overlap the inputs.
+ * Rows whose states are all empty come out empty (OUT = 0, LSE = -inf). */
+as_status as_compose(const float* outs, const float* lses, int n_states, int64_t rows, int d,
+                     int64_t state_stride_out, int64_t state_stride_lse,
+                     float* out, float* lse, void* stream);
+
+/* State cache: one entry per (query partition i, KV partition j), stored as
+ * P planes [P][B,H,S,d] (OUT) and [P][B,H,S] (LSE) in a caller-owned device
+ * buffer; entry (i, j) is plane j at the rows of partition i.  The host-side
+ * t_c[i*P+j] is the step of the entry's last store (-1 = never stored).
+ * The struct is caller-owned host memory; initialise it with as_cache_init. */
+typedef struct as_cache {
+  uint32_t magic;
+  int B, H, S, d, P;
+  as_dtype cache_dt;
+  float* out_planes;  /* device, [P][B,H,S,d] */
+  float* lse_planes;  /* device, [P][B,H,S] */
+  int32_t t_c[AS_MAX_P * AS_MAX_P];
+} as_cache;
+
+/* Bytes of device memory a cache for these sizes needs (fp32 states only:
+ * cache_dt must be AS_F32).  Returns 0 for invalid sizes. */
+size_t as_cache_bytes(int B, int H, int S, int d, int P, as_dtype cache_dt);
+
+/* Carve a cache out of `buf` (device, >= as_cache_bytes, 256-byte aligned)
+ * and mark every entry empty.  No device access happens here. */
+as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P,
+                        as_dtype cache_dt);
+
+/* Check a plan against the cache and derive the reuse bookkeeping, on the host
+ * only (no launch, no state change).  h_plan [P*P] row-major (row = query
+ * partition).  h_hit[i*P+j] = 1 for reused pairs, else 0; h_age[i*P+j] =
+ * step - t_c for reused pairs, else 0.  AS_ERR_CACHE_MISS if a reused entry
+ * was never stored; AS_ERR_INVALID_ARG for a code other than 0/1/2. */
+as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step,
+                          uint8_t* h_hit, int32_t* h_age);
+
+/* One denoising step's attention under a compute/reuse plan (DiTango review:
+ * Core claim; Referee Report, Summary).
+ *   final(i) = compose({AS_step(i,j) : plan fresh} U {C(i,j) : plan reuse})
+ * written to out [B,H,S,d], lse [B,H,S]; then for AS_PLAN_FRESH_STORE pairs
+ * C(i,j) <- AS_step(i,j) (device, in stream order) and t_c(i,j) <- step (host,
+ * at return).  h_hit / h_age (may be NULL) as in as_plan_resolve.  The plan is
+ * checked before any launch: on AS_ERR_CACHE_MISS or AS_ERR_INVALID_ARG
+ * nothing is launched and the cache is unchanged.  The cache must have been
+ * initialised for the same B, H, S, d, P. */
+as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
+                  const uint8_t* h_plan, int step, float* out, float* lse,
+                  uint8_t* h_hit, int32_t* h_age, void* stream);
+
+/* Synchronise `stream`, then read and clear the device error word that the
+ * kernels' bounded waits set.  *h_bits receives the raw bits (may be NULL).
+ * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, else AS_OK. */
+as_status as_device_status(void* stream, uint32_t* h_bits);
+
+/* Test hook for failure detection: launches one CTA that waits, with a poll
+ * budget of `poll_budget`, on a barrier that nothing completes.  The wait runs
+ * out, sets the device error word and the kernel returns; the context stays
+ * usable.  Read the outcome with as_device_status. */
+as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AS_PARTITION_H */
