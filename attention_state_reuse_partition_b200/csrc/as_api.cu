@@ -256,6 +256,14 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
     }
   }
   for (int j = 0; j < P; ++j) L.dest_of[j] = static_cast<int8_t>(j);
+  // every query partition reads the same KV list: one block of S rows, so
+  // query tiles are not cut at partition boundaries
+  bool uniform = true;
+  for (int i = 1; i < P && uniform; ++i) uniform = std::memcmp(h_plan, h_plan + i * P, P) == 0;
+  if (uniform) {
+    L.n_blocks = 1;
+    L.block_rows = S;
+  }
   L.out = out;
   L.lse = lse;
   L.out_rows = S;

@@ -1,23 +1,31 @@
 // Partition attention on the sm_100a tensor cores (bf16 in, fp32 state out).
 //
 // Computes attention states of DiTango (arXiv 2607.15650; review page,
-// "What carries the argument"): for a 128-row query tile and a list of KV
+// "What carries the argument"): for the query rows of a CTA and a list of KV
 // token ranges it runs the blockwise online softmax over 128-key tiles and
 // emits (OUT, LSE) per accumulation group -- the composite of every code-1
 // partition (the composition of Eq. 1-2 done on chip) and one state per
 // code-2 partition.
 //
-// One CTA per (query tile, head).  Warp roles:
-//   warp 0     TMA producer: Q once, then K and V tiles into 2-stage rings
-//   warp 1     TMEM allocator and UMMA issuer (one elected lane)
-//   warps 4-7  softmax: thread r owns query row r of the tile (TMEM lane r)
-// TMEM: S double buffer in columns [0,128) and [128,256), O in [256,256+D).
-// S = Q K^T and O += P V are tcgen05.mma kind::f16 (M=128, N=128 / D, K=16)
-// with operands in 128-byte-swizzled shared memory; P goes through shared
-// memory as bf16.  The issue order S_0, S_1, PV_0, S_2, PV_1, ... lets the
-// tensor core compute S_{j+1} and PV_{j-1} while the softmax warps work on S_j.
-// O is rescaled only when a row maximum grows by more than 2^8, which keeps
-// the result exact (OUT and the row sum share the same reference maximum).
+// One CTA per (256 query rows, head): two 128-row query tiles Q0, Q1 share
+// every K/V tile.  Warp roles:
+//   warp 0      TMA producer: Q0 and Q1 once, then K and V tiles (2-stage rings)
+//   warp 1      TMEM allocator and UMMA issuer (one elected lane)
+//   warps 4-7   softmax of Q0, warps 8-11 softmax of Q1: thread r owns row r of
+//               its tile (TMEM lane r)
+// TMEM columns: S_t = Q_t K^T at [128 t, 128 t + 128) (fp32), overwritten in
+// place by P_t (bf16 pairs, 64 columns) once the softmax has read it; O_t at
+// [256 + D t, 256 + D t + D).  S = Q K^T is an SS MMA (both operands in
+// 128-byte-swizzled shared memory), O += P V a TS MMA (P from TMEM, V from
+// shared memory, MN-major).  Issue order per KV tile j:
+//   PV0_j, QK0_{j+1}, PV1_j, QK1_{j+1}
+// so the tensor core runs one tile's PV and next QK (1024 cycles at d = 128)
+// while the other tile's softmax works.  A commit after QK_t completes only
+// when every earlier MMA has, so when the softmax of tile t sees S_t its
+// previous PV has finished: O_t may be rescaled and P_t written without a
+// further wait.  O is rescaled only when a row maximum grows by more than 2^8;
+// OUT and the row sum share the same reference maximum, so the result is
+// unchanged.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -26,43 +34,51 @@
 namespace asp {
 namespace {
 
-constexpr int BM = 128;       // query rows per tile
-constexpr int BN = 128;       // keys per KV tile
-constexpr int NST = 2;        // K and V ring depth
+constexpr int NQ = 2;          // query tiles per CTA
+constexpr int BM = 128;        // rows per query tile
+constexpr int BN = 128;        // keys per KV tile
+constexpr int NST = 2;         // K and V ring depth
 constexpr int REGION = 128 * 128;  // one 64-column bf16 chunk of a 128-row tile (bytes)
-constexpr int NTHREADS = 256;
+constexpr int NTHREADS = 128 * (1 + NQ);
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_O = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
+// registers: launched at LAUNCH_REGS per thread; the control warpgroup (TMA,
+// MMA, two idle warps) gives up registers to the softmax warpgroups.
+// 128 * CTRL_REGS + 128 * NQ * SOFTMAX_REGS == NTHREADS * LAUNCH_REGS
+constexpr int LAUNCH_REGS = 168;
+constexpr int CTRL_REGS = 72;
+constexpr int SOFTMAX_REGS = 216;
+static_assert(128 * CTRL_REGS + 128 * NQ * SOFTMAX_REGS == NTHREADS * LAUNCH_REGS, "register split");
 
 template <int D>
 struct Layout {
   static constexpr int NREG = D / 64;                 // 64-column chunks per row
-  static constexpr int TILE_BYTES = 128 * D * 2;      // Q, K or V tile
+  static constexpr int TILE_BYTES = 128 * D * 2;      // one Q, K or V tile
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE_BYTES;
+  static constexpr int K_OFF = Q_OFF + NQ * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + NST * TILE_BYTES;
-  static constexpr int P_OFF = V_OFF + NST * TILE_BYTES;
-  static constexpr int CTRL_OFF = P_OFF + BM * BN * 2;
+  static constexpr int CTRL_OFF = V_OFF + NST * TILE_BYTES;
+  static constexpr uint32_t O_COL = 256;              // O_t at O_COL + t * D
 };
 
 struct Ctrl {
   uint64_t q_full;
   uint64_t k_full[NST], k_empty[NST];
   uint64_t v_full[NST], v_empty[NST];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full;
-  uint64_t o_ready;
-  uint64_t o_free;
+  uint64_t s_full[NQ], p_full[NQ], o_ready[NQ], o_free[NQ];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int n_tiles;
   KvSchedule sched;
 };
 
 template <int D>
 constexpr int smem_bytes() {
-  return Layout<D>::CTRL_OFF + static_cast<int>(sizeof(Ctrl)) + 1024;
+  // at least 116 KB so that only one CTA (and one 512-column TMEM allocation)
+  // fits on an SM
+  constexpr int need = Layout<D>::CTRL_OFF + static_cast<int>(sizeof(Ctrl)) + 1024;
+  return need > 116 * 1024 ? need : 116 * 1024;
 }
 
 // Walks the tiles of a schedule in order, the same way in every role.
@@ -76,9 +92,7 @@ struct TileWalk {
     t = s->n_groups > 0 ? s->range_lo[r] : 0;
   }
   __device__ bool valid() const { return g < s->n_groups; }
-  __device__ bool first() const {
-    return r == s->group_first[g] && t == s->range_lo[r];
-  }
+  __device__ bool first() const { return r == s->group_first[g] && t == s->range_lo[r]; }
   __device__ bool last() const {
     return r == s->group_first[g] + s->group_count[g] - 1 && t + BN >= s->range_hi[r];
   }
@@ -99,11 +113,24 @@ struct TileWalk {
   }
 };
 
+__device__ int count_tiles(const KvSchedule& s) {
+  int n = 0;
+  for (int r = 0; r < s.n_ranges; ++r) n += (s.range_hi[r] - s.range_lo[r] + BN - 1) / BN;
+  return n;
+}
+
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint32_t budget) {
   for (uint32_t it = 0; it < budget; ++it)
     if (mbar_try_wait(bar, parity)) return true;
   raise_dev_error(AS_DEVERR_TIMEOUT);
   return false;
+}
+
+// all lanes of a warp wait; the result is the same in every lane
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t budget) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, budget);
+  return __all_sync(0xffffffffu, ok);
 }
 
 template <int D>
@@ -118,13 +145,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tiles_per_block = (L.block_rows + BM - 1) / BM;
+  const int tiles_per_block = (L.block_rows + NQ * BM - 1) / (NQ * BM);
   const int blk = blockIdx.x / tiles_per_block;
   const int qt = blockIdx.x % tiles_per_block;
   const int bh = blockIdx.y;
   const int block_lo = L.block_row0 + blk * L.block_rows;
-  const int q_lo = block_lo + qt * BM;
-  const int q_hi = min(min(q_lo + BM, block_lo + L.block_rows), L.S);
+  const int q_lo = block_lo + qt * NQ * BM;
+  const int q_hi = min(block_lo + L.block_rows, L.S);  // rows at or beyond q_hi are not written
   const uint32_t budget = L.poll_budget;
 
   if (threadIdx.x == 0) {
@@ -135,16 +162,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&c.v_full[s], 1);
       mbar_init(&c.v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&c.s_full[b], 1);
-      mbar_init(&c.s_free[b], 128);
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(&c.s_full[t], 1);
+      mbar_init(&c.p_full[t], 128);
+      mbar_init(&c.o_ready[t], 1);
+      mbar_init(&c.o_free[t], 128);
     }
-    mbar_init(&c.p_full, 128);
-    mbar_init(&c.o_ready, 1);
-    mbar_init(&c.o_free, 128);
     mbar_init(&c.drain, 1);
     c.abort = 0;
     build_schedule(L.code + blk * L.P, L.dest_of, L.P, L.n, c.sched);
+    c.n_tiles = count_tiles(c.sched);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -155,19 +182,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
+  const int n_tiles = c.n_tiles;
 
-  uint8_t* sQ = smem + Lay::Q_OFF;
-  uint8_t* sP = smem + Lay::P_OFF;
-
+  if (warp < 4) {
+  regs_dealloc<CTRL_REGS>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && c.sched.n_groups > 0) {
+    if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&c.q_full, Lay::TILE_BYTES);
-      for (int rg = 0; rg < Lay::NREG; ++rg)
-        tma_load_3d(sQ + rg * REGION, &tm_q, &c.q_full, rg * 64, q_lo, bh);
+      mbar_arrive_expect_tx(&c.q_full, NQ * Lay::TILE_BYTES);
+      for (int t = 0; t < NQ; ++t)
+        for (int rg = 0; rg < Lay::NREG; ++rg)
+          tma_load_3d(smem + Lay::Q_OFF + t * Lay::TILE_BYTES + rg * REGION, &tm_q, &c.q_full, rg * 64,
+                      q_lo + t * BM, bh);
       TileWalk w;
       int j = 0;
       for (w.start(&c.sched); w.valid(); w.next(), ++j) {
@@ -195,77 +224,79 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0 && c.sched.n_groups > 0) {
+    if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t p_base = smem_u32(sP);
-      bool ok = mbar_wait(&c.q_full, 0, abort_flag, budget);
-      tc_fence_after();
-      // the PV of tile j-1 is issued after the QK of tile j
-      int prev_st = 0, prev_group = 0;
-      bool prev_first = false;
-      int group = 0;
-      auto issue_pv = [&](int jp) -> bool {
-        if (prev_first && prev_group > 0)
-          if (!mbar_wait(&c.o_free, (prev_group - 1) & 1, abort_flag, budget)) return false;
-        if (!mbar_wait(&c.p_full, jp & 1, abort_flag, budget)) return false;
-        if (!mbar_wait(&c.v_full[prev_st], (jp / NST) & 1, abort_flag, budget)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + Lay::V_OFF + prev_st * Lay::TILE_BYTES);
+      const uint32_t q_base = smem_u32(smem + Lay::Q_OFF);
+      auto issue_qk = [&](int t, int j) {
+        const uint32_t k_base = smem_u32(smem + Lay::K_OFF + (j % NST) * Lay::TILE_BYTES);
+        const uint32_t qb = q_base + t * Lay::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(p_base + (kk >> 2) * REGION + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = smem_desc_sw128(v_base + kk * 16 * 128, REGION, 1024);
-          umma_bf16_ss(tmem + TMEM_O, a, b, IDESC_PV, (kk > 0 || !prev_first) ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * REGION + (kk & 3) * 32;
+          umma_bf16_ss(tmem + t * BN, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
+                       IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&c.o_ready);
-        umma_commit(&c.v_empty[prev_st]);
-        return true;
+        umma_commit(&c.s_full[t]);
       };
-      TileWalk w;
-      int j = 0;
-      if (ok) {
-        for (w.start(&c.sched); w.valid(); w.next(), ++j) {
-          const int st = j % NST;
-          if (!mbar_wait(&c.k_full[st], (j / NST) & 1, abort_flag, budget)) { ok = false; break; }
-          if (j >= 2 && !mbar_wait(&c.s_free[j & 1], ((j - 2) >> 1) & 1, abort_flag, budget)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(smem + Lay::K_OFF + st * Lay::TILE_BYTES);
-          const uint32_t s_col = (j & 1) * BN;
+      auto issue_pv = [&](int t, int j, bool first) {
+        const uint32_t v_base = smem_u32(smem + Lay::V_OFF + (j % NST) * Lay::TILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * REGION + (kk & 3) * 32;
-            const uint64_t a = smem_desc_sw128(q_base + off, 16, 1024);
-            const uint64_t b = smem_desc_sw128(k_base + off, 16, 1024);
-            umma_bf16_ss(tmem + s_col, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts(tmem + Lay::O_COL + t * D, tmem + t * BN + kk * 8,
+                       smem_desc_sw128(v_base + kk * 16 * 128, REGION, 1024), IDESC_PV,
+                       (kk > 0 || !first) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&c.q_full, 0, abort_flag, budget) && mbar_wait(&c.k_full[0], 0, abort_flag, budget);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < NQ; ++t) issue_qk(t, 0);
+        umma_commit(&c.k_empty[0]);
+        TileWalk w;
+        int j = 0, group = 0;
+        for (w.start(&c.sched); w.valid() && ok; w.next(), ++j) {
+          const bool first = w.first(), last = w.last();
+          if (first && j > 0) ++group;
+          const bool has_next = j + 1 < n_tiles;
+          const int st = j % NST;
+          for (int t = 0; t < NQ && ok; ++t) {
+            if (first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget)) ok = false;
+            if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag, budget)) ok = false;
+            if (ok && t == 0 && !mbar_wait(&c.v_full[st], (j / NST) & 1, abort_flag, budget)) ok = false;
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, j, first);
+            if (last) umma_commit(&c.o_ready[t]);
+            if (t == NQ - 1) umma_commit(&c.v_empty[st]);
+            if (has_next) {
+              if (t == 0 && !mbar_wait(&c.k_full[(j + 1) % NST], ((j + 1) / NST) & 1, abort_flag, budget)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_qk(t, j + 1);
+              if (t == NQ - 1) umma_commit(&c.k_empty[(j + 1) % NST]);
+            }
           }
-          umma_commit(&c.s_full[j & 1]);
-          umma_commit(&c.k_empty[st]);
-          if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
-          if (w.first() && j > 0) ++group;
-          prev_st = st;
-          prev_first = w.first();
-          prev_group = group;
         }
-        if (ok && j >= 1) issue_pv(j - 1);
       }
       // all issued MMAs must be complete before TMEM is released
       umma_commit(&c.drain);
       drain_wait(&c.drain, 0, budget);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_alloc<SOFTMAX_REGS>();
     // ------------------------------------------------------------ softmax
-    const int quarter = warp - 4;
+    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
+    const int quarter = warp & 3;           // TMEM lane quarter of this warp
     const int row = quarter * 32 + lane;
-    const int s_row = q_lo + row;
+    const int s_row = q_lo + t * BM + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t s_col = t * BN;
+    const uint32_t o_col = Lay::O_COL + t * D;
     const float sl2 = L.scale * 1.4426950408889634f;
     float m = -INFINITY, l = 0.f;
-    int pv_done = 0;
     int group = 0;
     TileWalk w;
     int j = 0;
@@ -274,27 +305,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const bool last = w.last();
       const int nv = w.nvalid();
       if (first && j > 0) ++group;
-      if (!mbar_wait(&c.s_full[j & 1], (j >> 1) & 1, abort_flag, budget)) break;
+      if (!warp_wait(&c.s_full[t], j & 1, abort_flag, budget)) break;
       tc_fence_after();
       float s[BN];
       {
-        uint32_t r[32];
+        uint32_t r[4][32];
 #pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          tmem_ld32(t_lane + (j & 1) * BN + ch * 32, r);
-          tmem_wait_ld();
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(t_lane + s_col + ch * 32, r[ch]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[ch * 32 + e] = __uint_as_float(r[e]);
-        }
+        for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[ch * 32 + e] = __uint_as_float(r[ch][e]);
       }
-      tc_fence_before();
-      mbar_arrive(&c.s_free[j & 1]);
-      float mx = -INFINITY;
+      if (nv < BN) {
 #pragma unroll
-      for (int e = 0; e < BN; ++e) {
-        if (e >= nv) s[e] = -INFINITY;
-        mx = fmaxf(mx, s[e]);
+        for (int e = 0; e < BN; ++e)
+          if (e >= nv) s[e] = -INFINITY;
       }
+      float mx8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx8[u] = s[u];
+#pragma unroll
+      for (int e = 8; e < BN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * sl2;
       float m_use = m, alpha = 1.f;
       bool rescale = false;
@@ -305,55 +340,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         alpha = ex2_approx(m - m_use);
         rescale = true;
       }
-      float rs = 0.f;
+      float rs8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
 #pragma unroll
       for (int e = 0; e < BN; ++e) {
         s[e] = ex2_approx(fmaf(s[e], sl2, -m_use));
-        rs += s[e];
+        rs8[e & 7] += s[e];
       }
-      // O and the P buffer are free once the previous PV has completed
-      bool ok = true;
-      while (pv_done < j) {
-        if (!mbar_wait(&c.o_ready, pv_done & 1, abort_flag, budget)) { ok = false; break; }
-        ++pv_done;
-      }
-      if (!ok) break;
-      tc_fence_after();
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      // the previous PV of this tile has completed (see the header), so O may
+      // be rescaled and P written over S now
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t r[32];
-          tmem_ld32(t_lane + TMEM_O + ch * 32, r);
+          tmem_ld32(t_lane + o_col + ch * 32, r);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(t_lane + TMEM_O + ch * 32, r);
+          tmem_st32(t_lane + o_col + ch * 32, r);
         }
-        tmem_wait_st();
       }
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[ch * 64 + 2 * e], s[ch * 64 + 2 * e + 1]);
+        tmem_st32(t_lane + s_col + ch * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&c.p_full[t]);
       l = first ? rs : fmaf(l, alpha, rs);
       m = m_use;
-      // P row -> shared memory, K-major 128-byte swizzle (two 64-key chunks)
-#pragma unroll
-      for (int ch = 0; ch < BN / 8; ++ch) {
-        uint4 pk;
-        pk.x = pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]);
-        pk.y = pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]);
-        pk.z = pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]);
-        pk.w = pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]);
-        const int region = ch >> 3;
-        const int phys = (ch & 7) ^ (row & 7);
-        *reinterpret_cast<uint4*>(sP + region * REGION + row * 128 + phys * 16) = pk;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&c.p_full);
       if (last) {
-        while (pv_done < j + 1) {
-          if (!mbar_wait(&c.o_ready, pv_done & 1, abort_flag, budget)) { ok = false; break; }
-          ++pv_done;
-        }
-        if (!ok) break;
+        if (!warp_wait(&c.o_ready[t], group & 1, abort_flag, budget)) break;
         tc_fence_after();
         const int dest = c.sched.group_dest[group];
         float* orow;
@@ -372,7 +394,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t r[32];
-          tmem_ld32(t_lane + TMEM_O + ch * 32, r);
+          tmem_ld32(t_lane + o_col + ch * 32, r);
           tmem_wait_ld();
           if (write) {
 #pragma unroll
@@ -385,7 +407,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         if (write) *lrow = (m + log2f(l)) * 0.6931471805599453f;
         tc_fence_before();
-        mbar_arrive(&c.o_free);
+        mbar_arrive(&c.o_free[t]);
       }
     }
     tc_fence_before();
@@ -435,7 +457,12 @@ cudaError_t launch_d(const AttnLaunch& L, cudaStream_t st) {
   constexpr int smem = smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int tiles_per_block = (L.block_rows + BM - 1) / BM;
+  // the in-kernel register split assumes exactly LAUNCH_REGS per thread at launch
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+  const int tiles_per_block = (L.block_rows + NQ * BM - 1) / (NQ * BM);
   dim3 grid(L.n_blocks * tiles_per_block, BH);
   attn_tc_kernel<D><<<grid, NTHREADS, smem, st>>>(tq, tk, tv, L);
   return cudaGetLastError();

@@ -70,51 +70,63 @@ def attn_flops(s) -> float:
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, power and clock-event reasons through NVML (read-only
+    queries) every 10 ms in a background thread.  Samples taken inside the
+    timed region are marked via ``mark_timed``."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, gpu_index: int, interval: float = 0.01):
+        import threading
+        self.gpu, self.interval = gpu_index, interval
+        self.samples = []
+        self.timed = False
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.error = None
+
+    def _run(self):
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByIndex(self.gpu)
+            smax = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            while not self.stop.is_set():
+                sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                try:
+                    reasons = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except AttributeError:
+                    reasons = N.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                power = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((self.timed, sm, smax, power, reasons))
+                time.sleep(self.interval)
+            N.nvmlShutdown()
+        except Exception as e:  # noqa: BLE001
+            self.error = repr(e)
 
     def __enter__(self):
-        try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        self.thread.start()
         return self
 
+    def mark_timed(self, on: bool):
+        self.timed = on
+
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.stop.set()
+        self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] not in ("", "[N/A]"))}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"no samples ({self.error})"]}
+        timed = [x for x in self.samples if x[0]]
+        use = timed if timed else self.samples
+        reasons = sorted({name for x in use for bit, name in self.REASONS.items() if x[4] & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": float(use[0][2]),
+                "reasons": reasons, "samples_timed": len(timed), "samples_total": len(self.samples),
+                "power_w_max": max(x[3] for x in use),
+                "how": "NVML every 10 ms; median over the samples inside the timed region "
+                       "(all samples, warm-up included, when the region is shorter than one interval)"}
 
 
 # ---------------------------------------------------------------------------
@@ -170,21 +182,28 @@ def run_own(args, rank, world, device):
     def step():
         api.as_step(cache, q, k, v, plan, 0, out=out, lse=lse)
 
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     with ClockSampler(torch.cuda.current_device()) as clk:
+        t_end = time.perf_counter() + args.warm_seconds   # warm the clocks up
+        done = 0
+        while done < args.warmup or time.perf_counter() < t_end:
+            flush.fill_(1.0)
+            step()
+            done += 1
+            if done % 16 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        clk.mark_timed(True)
         for i in range(args.steps):
             flush.fill_(float(i))           # L2 flush, keeps the GPU busy across the launch gap
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+        clk.mark_timed(False)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -198,6 +217,11 @@ def run_own(args, rank, world, device):
         ms_max = t.item()
     flops = attn_flops(s)
     value = flops * world / (ms_max * 1e-3) / 1e12
+
+    result = {"ms": ms, "ms_max": ms_max, "value": value, "flops": flops, "clocks": clk.summary(),
+              "gpu_launches": args.steps, "step_ms": times, "e2e": None}
+    if args.kernel_only:
+        return result, (q, k, v, s)
 
     # end to end through the public API with pinned host buffers
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
@@ -231,13 +255,8 @@ def run_own(args, rank, world, device):
     d2h = hout.numel() * 4 + hlse.numel() * 4
     assert torch.allclose(hout.to(device), out), "e2e output differs from the device-resident run"
 
-    result = {
-        "ms": ms, "ms_max": ms_max, "value": value, "flops": flops,
-        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "clocks": clk.summary(), "gpu_launches": args.steps,
-        "step_ms": times,
-    }
+    result["e2e"] = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     del cache, flush
     torch.cuda.empty_cache()
     return result, (q, k, v, s)
@@ -312,7 +331,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
     ap.add_argument("--no-secondary", action="store_true")
-    ap.add_argument("--cpu-sample-rows", type=int, default=48)
+    ap.add_argument("--warm-seconds", type=float, default=1.0,
+                    help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time the device-resident step only (no e2e, CPU baseline or secondary workloads)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -332,19 +354,19 @@ def main():
     peaks = load_peaks()
     res, (q, k, v, s) = run_own(args, rank, world, device)
     secondary = {}
-    if not args.no_secondary and world == 1:
+    if not args.no_secondary and not args.kernel_only and world == 1:
         comp = run_compose(args, device)
         comp["frac_of_hbm"] = comp["GB/s"] / peaks["hbm_gbs"]
         secondary["compose"] = comp
         secondary["reuse"] = run_reuse(args, device)
 
     cpu = None
-    if rank == 0 and world == 1:
-        heads = [0, 11, 23]
-        dt, fl = oracle_sample(s, q, k, v, args.cpu_sample_rows, heads)
+    if rank == 0 and world == 1 and not args.kernel_only:
+        heads = list(range(s.H))
+        dt, fl = oracle_sample(s, q, k, v, s.n, heads)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"{args.cpu_sample_rows} query rows per partition x {len(heads)} heads of {WORKLOAD}, "
-                         f"all {s.S} keys, float64 ({dt:.1f} s)"}
+               "sample": f"the whole {WORKLOAD} step (all {s.S} query rows x {s.H} heads, all {s.S} keys), "
+                         f"float64, one pass ({dt:.1f} s)"}
 
     ms = res["ms_max"]
     achieved = res["flops"] / (res["ms"] * 1e-3) / 1e12
@@ -362,6 +384,8 @@ def main():
                      "kernel": "attn_tc_kernel<128>", "peak_source": f"{peaks['source']} bf16 burst"},
         "e2e": res["e2e"], "clocks": res["clocks"], "gpu_launches": res["gpu_launches"],
     }
+    if line["e2e"] is None:
+        del line["e2e"]
     if cpu:
         line["cpu_baseline"] = cpu
     if secondary:
@@ -381,7 +405,7 @@ def run_reference(args, rank, world):
     s = W.spec(WORKLOAD)
     q, k, v = W.flux_qkv(s)
     heads = [0, 11, 23]
-    rows = 8
+    rows = s.n
     for _ in range(args.warmup):
         oracle_sample(s, q, k, v, rows, heads)
     tot_t, tot_f = 0.0, 0.0
@@ -390,12 +414,12 @@ def run_reference(args, rank, world):
         tot_t += dt
         tot_f += fl
     value = tot_f / tot_t / 1e12
-    sample = f"{rows} query rows per partition x {len(heads)} heads of {WORKLOAD}, all {s.S} keys, float64"
+    sample = f"per step: all {s.S} query rows x {len(heads)} of {s.H} heads of {WORKLOAD}, all {s.S} keys, float64"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{WORKLOAD}: B=1 H=24 S=4608 d=128, P=8, all pairs fresh (sampled rows)",
+        "config": {"workload": f"{WORKLOAD}: B=1 H=24 S=4608 d=128, P=8, all pairs fresh (3 heads per step)",
                    "global_batch": 1, "seq_len": s.S, "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
