@@ -21,7 +21,8 @@ STATUS_NAMES = {
 
 # every entry point declared in include/as_partition.h
 EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as_cache_bytes",
-           "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe")
+           "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe",
+           "as_debug_exp2")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -70,6 +71,8 @@ def _load() -> ctypes.CDLL:
     lib.as_device_status.argtypes = [vp, ctypes.POINTER(u32)]
     lib.as_debug_timeout_probe.restype = c_int
     lib.as_debug_timeout_probe.argtypes = [u32, vp]
+    lib.as_debug_exp2.restype = c_int
+    lib.as_debug_exp2.argtypes = [vp, vp, i64, c_int, vp]
     return lib
 
 

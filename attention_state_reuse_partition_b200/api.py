@@ -176,5 +176,12 @@ def as_device_status(stream=None) -> int:
     return bits.value
 
 
+def as_debug_exp2(x, mode: int = 0, stream=None):
+    """2^x on the device: mode 0 = FMA-pipe polynomial, 1 = MUFU ex2.approx."""
+    y = torch.empty_like(x)
+    check(LIB.as_debug_exp2(_dev(x, "x"), _dev(y, "y"), x.numel(), int(mode), _stream_ptr(stream)))
+    return y
+
+
 def as_debug_timeout_probe(poll_budget: int = 64, stream=None) -> None:
     check(LIB.as_debug_timeout_probe(int(poll_budget), _stream_ptr(stream)))

@@ -336,4 +336,15 @@ as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream) {
   return ok();
 }
 
+as_status as_debug_exp2(const float* x, float* y, int64_t n, int mode, void* stream) {
+  if (n < 0 || (mode != 0 && mode != 1) || (n > 0 && (!x || !y)))
+    return fail(AS_ERR_INVALID_ARG, "as_debug_exp2: bad arguments");
+  if (n == 0) return ok();
+  as_status s = check_device();
+  if (s != AS_OK) return s;
+  cudaError_t e = asp::launch_exp2_probe(x, y, n, mode, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 probe launch");
+  return ok();
+}
+
 }  // extern "C"

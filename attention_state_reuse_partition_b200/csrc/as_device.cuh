@@ -226,6 +226,63 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// exp2 on the FMA pipe, to relieve the MUFU unit (exp2_poly2 below).  2^x = 2^n * 2^f with
+// n = round(x) (by adding and subtracting 1.5 * 2^23) and f = x - n in
+// [-1/2, 1/2]; 2^f is a degree-4 minimax polynomial (relative error 2.7e-6,
+// coefficients from gen_exp2_poly.py) and 2^n is added to its exponent bits.
+// x is clamped below at -125 so the result stays a normal float (2^-125 is
+// negligible against a row maximum of 1).
+constexpr float EXP2_C0 = 9.999992847e-01f;
+constexpr float EXP2_C1 = 6.931217909e-01f;
+constexpr float EXP2_C2 = 2.402474433e-01f;
+constexpr float EXP2_C3 = 5.591785908e-02f;
+constexpr float EXP2_C4 = 9.570102207e-03f;
+constexpr float ROUND_MAGIC = 12582912.0f;  // 1.5 * 2^23
+
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (Blackwell f32x2 FMA-pipe instructions)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly on a pair, with the rounding and the polynomial in f32x2 form
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t = f2_add(x, f2_pack(ROUND_MAGIC, ROUND_MAGIC));
+  const uint64_t n = f2_add(t, f2_pack(-ROUND_MAGIC, -ROUND_MAGIC));
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);
+  uint64_t p = f2_fma(f2_pack(EXP2_C4, EXP2_C4), f, f2_pack(EXP2_C3, EXP2_C3));
+  p = f2_fma(p, f, f2_pack(EXP2_C2, EXP2_C2));
+  p = f2_fma(p, f, f2_pack(EXP2_C1, EXP2_C1));
+  p = f2_fma(p, f, f2_pack(EXP2_C0, EXP2_C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

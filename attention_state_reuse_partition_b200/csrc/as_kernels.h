@@ -71,6 +71,7 @@ cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st);
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st);
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st);
 cudaError_t launch_timeout_probe(unsigned int poll_budget, cudaStream_t st);
+cudaError_t launch_exp2_probe(const float* x, float* y, long long n, int mode, cudaStream_t st);
 cudaError_t read_and_clear_dev_error(unsigned int* bits, cudaStream_t st);
 
 }  // namespace asp

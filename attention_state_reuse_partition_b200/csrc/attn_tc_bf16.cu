@@ -17,13 +17,13 @@
 // place by P_t (bf16 pairs, 64 columns) once the softmax has read it; O_t at
 // [256 + D t, 256 + D t + D).  S = Q K^T is an SS MMA (both operands in
 // 128-byte-swizzled shared memory), O += P V a TS MMA (P from TMEM, V from
-// shared memory, MN-major).  Issue order per KV tile j:
-//   PV0_j, QK0_{j+1}, PV1_j, QK1_{j+1}
-// so the tensor core runs one tile's PV and next QK (1024 cycles at d = 128)
-// while the other tile's softmax works.  A commit after QK_t completes only
-// when every earlier MMA has, so when the softmax of tile t sees S_t its
-// previous PV has finished: O_t may be rescaled and P_t written without a
-// further wait.  O is rescaled only when a row maximum grows by more than 2^8;
+// shared memory, MN-major).  Per KV tile j the issuer sends, for t = 0, 1,
+// one uninterrupted burst PV_t,j + QK_t,j+1 (16 MMAs, 1024 cycles at d = 128,
+// all waits done before the burst, because the issuing thread runs only a few
+// MMAs ahead of the tensor core), so the tensor core works on one tile while
+// the other tile's softmax runs.  A commit after QK_t completes only when
+// every earlier MMA has, so when the softmax of tile t sees S_t its previous
+// PV has finished: O_t may be rescaled and P_t written without a further wait.  O is rescaled only when a row maximum grows by more than 2^8;
 // OUT and the row sum share the same reference maximum, so the result is
 // unchanged.
 #include <cuda.h>
@@ -42,12 +42,16 @@ constexpr int REGION = 128 * 128;  // one 64-column bf16 chunk of a 128-row tile
 constexpr int NTHREADS = 128 * (1 + NQ);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
+#ifndef ASP_POLY_PAIR_EVERY
+#define ASP_POLY_PAIR_EVERY 0
+#endif
+constexpr int POLY_PAIR_EVERY = ASP_POLY_PAIR_EVERY;  // every n-th pair of exponentials on the FMA pipe
 // registers: launched at LAUNCH_REGS per thread; the control warpgroup (TMA,
 // MMA, two idle warps) gives up registers to the softmax warpgroups.
 // 128 * CTRL_REGS + 128 * NQ * SOFTMAX_REGS == NTHREADS * LAUNCH_REGS
 constexpr int LAUNCH_REGS = 168;
-constexpr int CTRL_REGS = 72;
-constexpr int SOFTMAX_REGS = 216;
+constexpr int CTRL_REGS = 88;
+constexpr int SOFTMAX_REGS = 208;
 static_assert(128 * CTRL_REGS + 128 * NQ * SOFTMAX_REGS == NTHREADS * LAUNCH_REGS, "register split");
 
 template <int D>
@@ -81,34 +85,51 @@ constexpr int smem_bytes() {
   return need > 116 * 1024 ? need : 116 * 1024;
 }
 
-// Walks the tiles of a schedule in order, the same way in every role.
+// Walks the tiles of a schedule in order, the same way in every role.  The
+// bounds of the current range and group are cached in registers; shared
+// memory is read only when the walk enters a new range.
 struct TileWalk {
   const KvSchedule* s;
   int g, r, t;
+  int r_lo, r_hi, g_first_r, g_last_r, n_groups;
+  __device__ void load_range() {
+    r_lo = s->range_lo[r];
+    r_hi = s->range_hi[r];
+  }
+  __device__ void load_group() {
+    g_first_r = s->group_first[g];
+    g_last_r = g_first_r + s->group_count[g] - 1;
+  }
   __device__ void start(const KvSchedule* sched) {
     s = sched;
+    n_groups = s->n_groups;
     g = 0;
-    r = s->n_groups > 0 ? s->group_first[0] : 0;
-    t = s->n_groups > 0 ? s->range_lo[r] : 0;
+    if (n_groups > 0) {
+      load_group();
+      r = g_first_r;
+      load_range();
+      t = r_lo;
+    }
   }
-  __device__ bool valid() const { return g < s->n_groups; }
-  __device__ bool first() const { return r == s->group_first[g] && t == s->range_lo[r]; }
-  __device__ bool last() const {
-    return r == s->group_first[g] + s->group_count[g] - 1 && t + BN >= s->range_hi[r];
-  }
-  __device__ int nvalid() const { return min(BN, s->range_hi[r] - t); }
+  __device__ bool valid() const { return g < n_groups; }
+  __device__ bool first() const { return r == g_first_r && t == r_lo; }
+  __device__ bool last() const { return r == g_last_r && t + BN >= r_hi; }
+  __device__ int nvalid() const { return min(BN, r_hi - t); }
   __device__ void next() {
     t += BN;
-    if (t < s->range_hi[r]) return;
+    if (t < r_hi) return;
     ++r;
-    if (r < s->group_first[g] + s->group_count[g]) {
-      t = s->range_lo[r];
+    if (r <= g_last_r) {
+      load_range();
+      t = r_lo;
       return;
     }
     ++g;
-    if (g < s->n_groups) {
-      r = s->group_first[g];
-      t = s->range_lo[r];
+    if (g < n_groups) {
+      load_group();
+      r = g_first_r;
+      load_range();
+      t = r_lo;
     }
   }
 };
@@ -227,30 +248,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
-      const uint32_t q_base = smem_u32(smem + Lay::Q_OFF);
+      // descriptors of stage 0; stages, query tiles and k-steps only move the
+      // start address field (16-byte units), which stays below 2^14 for 227 KB
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + Lay::Q_OFF), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem + Lay::K_OFF), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + Lay::V_OFF), REGION, 1024);
+      constexpr uint32_t TILE16 = Lay::TILE_BYTES >> 4;
       auto issue_qk = [&](int t, int j) {
-        const uint32_t k_base = smem_u32(smem + Lay::K_OFF + (j % NST) * Lay::TILE_BYTES);
-        const uint32_t qb = q_base + t * Lay::TILE_BYTES;
+        const uint64_t dq = dq0 + t * TILE16;
+        const uint64_t dk = dk0 + (j % NST) * TILE16;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * REGION + (kk & 3) * 32;
-          umma_bf16_ss(tmem + t * BN, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
-                       IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * REGION + (kk & 3) * 32) >> 4;
+          umma_bf16_ss(tmem + t * BN, dq + off16, dk + off16, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&c.s_full[t]);
       };
       auto issue_pv = [&](int t, int j, bool first) {
-        const uint32_t v_base = smem_u32(smem + Lay::V_OFF + (j % NST) * Lay::TILE_BYTES);
+        const uint64_t dv = dv0 + (j % NST) * TILE16;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ts(tmem + Lay::O_COL + t * D, tmem + t * BN + kk * 8,
-                       smem_desc_sw128(v_base + kk * 16 * 128, REGION, 1024), IDESC_PV,
-                       (kk > 0 || !first) ? 1u : 0u);
+          umma_bf16_ts(tmem + Lay::O_COL + t * D, tmem + t * BN + kk * 8, dv + ((kk * 16 * 128) >> 4),
+                       IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
       };
       bool ok = mbar_wait(&c.q_full, 0, abort_flag, budget) && mbar_wait(&c.k_full[0], 0, abort_flag, budget);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < NQ; ++t) issue_qk(t, 0);
+        for (int t = 0; t < NQ; ++t) {
+          issue_qk(t, 0);
+          umma_commit(&c.s_full[t]);
+        }
         umma_commit(&c.k_empty[0]);
         TileWalk w;
         int j = 0, group = 0;
@@ -259,23 +285,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (first && j > 0) ++group;
           const bool has_next = j + 1 < n_tiles;
           const int st = j % NST;
-          for (int t = 0; t < NQ && ok; ++t) {
+          for (int t = 0; t < NQ; ++t) {
+            // every wait of the burst first, then the 16 MMAs back to back
             if (first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget)) ok = false;
             if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag, budget)) ok = false;
             if (ok && t == 0 && !mbar_wait(&c.v_full[st], (j / NST) & 1, abort_flag, budget)) ok = false;
+            if (ok && t == 0 && has_next &&
+                !mbar_wait(&c.k_full[(j + 1) % NST], ((j + 1) / NST) & 1, abort_flag, budget))
+              ok = false;
             if (!ok) break;
             tc_fence_after();
             issue_pv(t, j, first);
+            if (has_next) issue_qk(t, j + 1);
             if (last) umma_commit(&c.o_ready[t]);
-            if (t == NQ - 1) umma_commit(&c.v_empty[st]);
-            if (has_next) {
-              if (t == 0 && !mbar_wait(&c.k_full[(j + 1) % NST], ((j + 1) / NST) & 1, abort_flag, budget)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              issue_qk(t, j + 1);
-              if (t == NQ - 1) umma_commit(&c.k_empty[(j + 1) % NST]);
+            if (has_next) umma_commit(&c.s_full[t]);
+            if (t == NQ - 1) {
+              umma_commit(&c.v_empty[st]);
+              if (has_next) umma_commit(&c.k_empty[(j + 1) % NST]);
             }
           }
         }
@@ -323,14 +349,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int e = 0; e < BN; ++e)
           if (e >= nv) s[e] = -INFINITY;
       }
-      float mx8[8];
+      // row maximum: four independent chains of 3-input max
+      float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = s[u];
-#pragma unroll
-      for (int e = 8; e < BN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_tile = mx * sl2;
+      for (int e = 4; e < BN; e += 8) {
+        mx4[0] = max3(mx4[0], s[e + 0], s[e + 1]);
+        mx4[1] = max3(mx4[1], s[e + 2], s[e + 3]);
+        mx4[2] = max3(mx4[2], s[e + 4], s[e + 5]);
+        if (e + 7 < BN) mx4[3] = max3(mx4[3], s[e + 6], s[e + 7]);
+      }
+      const float m_tile = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
       float m_use = m, alpha = 1.f;
       bool rescale = false;
       if (first) {
@@ -340,15 +368,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         alpha = ex2_approx(m - m_use);
         rescale = true;
       }
-      float rs8[8];
+      // p = 2^(s * scale * log2 e - m): scale-subtract and row sum on packed
+      // pairs; one pair in POLY_PAIR_EVERY evaluated on the FMA pipe
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_use, -m_use);
+      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[BN / 2];  // P as bf16 pairs, written to TMEM over S
 #pragma unroll
-      for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
-#pragma unroll
-      for (int e = 0; e < BN; ++e) {
-        s[e] = ex2_approx(fmaf(s[e], sl2, -m_use));
-        rs8[e & 7] += s[e];
+      for (int i = 0; i < BN / 2; ++i) {
+        const uint64_t x2 = f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2x2, negm2);
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        uint64_t p2;
+        if (POLY_PAIR_EVERY > 0 && i % POLY_PAIR_EVERY == POLY_PAIR_EVERY - 1)
+          p2 = exp2_poly2(x0, x1);
+        else
+          p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        sum2[i & 3] = f2_add(sum2[i & 3], p2);
+        float p0, p1;
+        f2_unpack(p2, p0, p1);
+        pk[i] = pack_bf16x2(p0, p1);
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      float rs;
+      {
+        const uint64_t a = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+        float lo, hi;
+        f2_unpack(a, lo, hi);
+        rs = lo + hi;
+      }
       // the previous PV of this tile has completed (see the header), so O may
       // be rescaled and P written over S now
       if (__any_sync(0xffffffffu, rescale)) {
@@ -362,13 +409,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tmem_st32(t_lane + o_col + ch * 32, r);
         }
       }
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[ch * 64 + 2 * e], s[ch * 64 + 2 * e + 1]);
-        tmem_st32(t_lane + s_col + ch * 32, pk);
-      }
+      tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&c.p_full[t]);
@@ -481,7 +523,24 @@ __global__ void timeout_probe_kernel(unsigned int budget) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, budget);
 }
 
+__global__ void exp2_probe_kernel(const float* x, float* y, long long n, int mode) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+  {
+    float lo = 0.f, hi = 0.f;
+    if (mode == 0) f2_unpack(exp2_poly2(x[i], x[i]), lo, hi);
+    y[i] = mode == 0 ? lo : ex2_approx(x[i]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_probe(const float* x, float* y, long long n, int mode, cudaStream_t st) {
+  const long long blocks = (n + 255) / 256;
+  exp2_probe_kernel<<<static_cast<unsigned>(blocks < 4096 ? (blocks > 0 ? blocks : 1) : 4096), 256, 0, st>>>(
+      x, y, n, mode);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_timeout_probe(unsigned int poll_budget, cudaStream_t st) {
   timeout_probe_kernel<<<1, 32, 0, st>>>(poll_budget);

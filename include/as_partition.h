@@ -150,6 +150,12 @@ as_status as_device_status(void* stream, uint32_t* h_bits);
  * usable.  Read the outcome with as_device_status. */
 as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream);
 
+/* Test hook for the two exp2 evaluations the attention kernel mixes:
+ * y[i] = 2^x[i] for n device floats, mode 0 = the FMA-pipe polynomial
+ * (range reduction to [-1/2, 1/2], degree-4 minimax fit, relative error
+ * <= 3e-6, inputs clamped below at -125), mode 1 = the MUFU ex2.approx. */
+as_status as_debug_exp2(const float* x, float* y, int64_t n, int mode, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -267,3 +267,18 @@ def test_timeout_is_reported_and_context_survives(api):
     out, lse = api.as_compose(outs, lses)
     ref_o, ref_l = O.compose([(f64(outs[k]), f64(lses[k])) for k in range(3)])
     check_f32(out, lse, ref_o, ref_l, "after timeout")
+
+
+# ---------------------------------------------------------------------------
+# the two exp2 evaluations mixed in the softmax, against CUDA's exp2
+# ---------------------------------------------------------------------------
+
+def test_exp2_paths_against_cuda(api):
+    x = torch.linspace(-124.9, 9.0, 1 << 22, device="cuda")
+    ref = torch.exp2(x.double())
+    for mode, tol in ((0, 4e-6), (1, 2e-6)):
+        y = api.as_debug_exp2(x, mode).double()
+        rel = ((y / ref) - 1).abs().max().item()
+        assert rel < tol, (mode, rel)
+    masked = api.as_debug_exp2(torch.tensor([-math.inf, -200.0], device="cuda"), 0)
+    assert torch.all(masked > 0) and torch.all(masked < 3e-38)
