@@ -286,13 +286,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const bool has_next = j + 1 < n_tiles;
           const int st = j % NST;
           for (int t = 0; t < NQ; ++t) {
-            // every wait of the burst first, then the 16 MMAs back to back
-            if (first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget)) ok = false;
-            if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag, budget)) ok = false;
-            if (ok && t == 0 && !mbar_wait(&c.v_full[st], (j / NST) & 1, abort_flag, budget)) ok = false;
+            // every wait of the burst first (the data waits, satisfied early,
+            // before the softmax handshake), then the 16 MMAs back to back
+            if (t == 0 && !mbar_wait(&c.v_full[st], (j / NST) & 1, abort_flag, budget)) ok = false;
             if (ok && t == 0 && has_next &&
                 !mbar_wait(&c.k_full[(j + 1) % NST], ((j + 1) / NST) & 1, abort_flag, budget))
               ok = false;
+            if (ok && first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget))
+              ok = false;
+            if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag, budget)) ok = false;
             if (!ok) break;
             tc_fence_after();
             issue_pv(t, j, first);
