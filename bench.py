@@ -61,8 +61,56 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+CSRC = os.path.join(ROOT, "attention_state_reuse_partition_b200", "csrc")
+KERNEL_SOURCES = {
+    "attn_tc_kernel<128>": ("attn_tc_bf16.cu", "as_device.cuh", "as_kernels.h"),
+    "compose_strided_kernel<128>": ("compose.cu", "as_device.cuh", "as_kernels.h"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """First 16 hex digits of the SHA-256 of the sources a kernel is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, units_scale: float = 1.0):
+    """DRAM bytes (read + write) per launch from the committed ncu summary
+    (profiles/ncu_traffic.txt), scaled by units_scale when the capture ran a
+    smaller case; None if absent or if the kernel's sources changed since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entry = json.load(f).get(kernel)
+    if not entry or entry.get("source_sha256_16") != kernel_source_hash(kernel):
+        return None
+    return entry["dram_bytes_per_launch"] * units_scale
+
+
 def attn_flops(s) -> float:
     return 4.0 * s.B * s.H * s.S * s.S * s.d
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of a per-rank scalar over all ranks (identity at one rank).
+    Every rank must call it at the same point (a collective)."""
+    if not torch.distributed.is_available() or not torch.distributed.is_initialized() \
+            or torch.distributed.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed units_per_rank in at most
+    ms_max milliseconds (the slowest rank's time)."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -210,13 +258,9 @@ def run_own(args, rank, world, device):
     times = [a.elapsed_time(b) for a, b in ev]
     ms = sum(times) / len(times)
     api.as_device_status()
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = t.item()
+    ms_max = max_over_ranks(ms, device)
     flops = attn_flops(s)
-    value = flops * world / (ms_max * 1e-3) / 1e12
+    value = weak_scaling_value(flops, world, ms_max) / 1e12
 
     result = {"ms": ms, "ms_max": ms_max, "value": value, "flops": flops, "clocks": clk.summary(),
               "gpu_launches": args.steps, "step_ms": times, "e2e": None}
@@ -246,27 +290,34 @@ def run_own(args, rank, world, device):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = hout.numel() * 4 + hlse.numel() * 4
     assert torch.allclose(hout.to(device), out), "e2e output differs from the device-resident run"
 
-    result["e2e"] = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    result["e2e"] = {"value": weak_scaling_value(flops, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     del cache, flush
     torch.cuda.empty_cache()
     return result, (q, k, v, s)
 
 
+def ncu_compose_rows() -> int:
+    """Rows of the compose case the committed ncu capture ran (196608)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if os.path.exists(path):
+        with open(path) as f:
+            e = json.load(f).get("compose_strided_kernel<128>")
+        if e:
+            return int(e.get("rows", 196608))
+    return 196608
+
+
 def run_compose(args, device):
     """Compose-bound workload: 32 fp32 states per row merged into one."""
     from attention_state_reuse_partition_b200 import api
     s = W.spec("compose_bound")
-    outs, lses = W.compose_states(s, device=device)
+    outs, lses = W.compose_states(s, device=device, rows=args.compose_rows)
     out = torch.empty(outs.shape[1:], device=device)
     lse = torch.empty(lses.shape[1:], device=device)
     for _ in range(3):
@@ -324,6 +375,40 @@ def run_reuse(args, device):
             "reuse_mse_vs_full": mse}
 
 
+def run_video_long(args, device):
+    """Long video trajectory: an anchor step, then three reuse steps (window 4,
+    a seeded 10% of reused pairs forced fresh and stored each step)."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec("video_long")
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    out = torch.empty((s.B, s.H, s.S, s.d), device=device)
+    lse = torch.empty((s.B, s.H, s.S), device=device)
+    per_step = []
+    last = None
+    for t, q, k, v in W.video_trajectory(s, device=device):
+        plan = W.plan_for_step(s, t).numpy()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        api.as_step(cache, q, k, v, plan, t, out=out, lse=lse)
+        b.record()
+        torch.cuda.synchronize()
+        n_fresh = int((plan != W.PLAN_REUSE).sum())
+        n_reuse = int((plan == W.PLAN_REUSE).sum())
+        n_store = int((plan == W.PLAN_FRESH_STORE).sum())
+        ms = a.elapsed_time(b)
+        fl = 4.0 * s.B * s.H * n_fresh * s.n * s.n * s.d
+        per_step.append({"step": t, "ms": round(ms, 3), "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
+                         "stored_pairs": n_store, "fresh_tflops_whole_step": round(fl / (ms * 1e-3) / 1e12, 1)})
+        last = (q, k, v)
+    q, k, v = last
+    full_o, _ = api.as_partition_attn(q, k, v, s.P, -1, list(range(s.P)))
+    torch.cuda.synchronize()
+    mse = torch.mean((out - full_o) ** 2).item()
+    del cache, full_o, out, lse, last, q, k, v
+    torch.cuda.empty_cache()
+    return {"workload": "video_long (4 steps)", "steps": per_step, "reuse_mse_vs_full_last_step": mse}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -333,6 +418,10 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
+    ap.add_argument("--only", choices=["compose", "reuse", "video_long"], default=None,
+                    help="run one secondary workload alone and print its JSON (for profiling)")
+    ap.add_argument("--compose-rows", type=int, default=None,
+                    help="rows of the compose workload (default: all B*H*S rows)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device-resident step only (no e2e, CPU baseline or secondary workloads)")
     args = ap.parse_args()
@@ -347,6 +436,10 @@ def main():
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.only is not None:
+        fn = {"compose": run_compose, "reuse": run_reuse, "video_long": run_video_long}[args.only]
+        print(json.dumps({"only": args.only, **fn(args, device)}))
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -357,8 +450,11 @@ def main():
     if not args.no_secondary and not args.kernel_only and world == 1:
         comp = run_compose(args, device)
         comp["frac_of_hbm"] = comp["GB/s"] / peaks["hbm_gbs"]
+        rows_full = W.spec("compose_bound").B * W.spec("compose_bound").H * W.spec("compose_bound").S
+        comp["traffic"] = measured_traffic("compose_strided_kernel<128>", rows_full / ncu_compose_rows())
         secondary["compose"] = comp
         secondary["reuse"] = run_reuse(args, device)
+        secondary["video_long"] = run_video_long(args, device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.kernel_only:
@@ -380,7 +476,7 @@ def main():
                    "parallelism": f"replicas{world}" if world > 1 else "single", "l2": "flushed (256 MiB write) "
                    "before every timed step"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic("attn_tc_kernel<128>"),
                      "kernel": "attn_tc_kernel<128>", "peak_source": f"{peaks['source']} bf16 burst"},
         "e2e": res["e2e"], "clocks": res["clocks"], "gpu_launches": res["gpu_launches"],
     }

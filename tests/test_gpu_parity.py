@@ -202,6 +202,19 @@ def test_step_video_reuse_full(api):
     _run_steps(api, s, steps, plans, rows=W.sample_rows(s, 8).numpy(), heads=[0, 13, 23])
 
 
+def test_step_video_long_full(api):
+    """The long-trajectory workload at full size (S=65536, H=40, P=32, 4 steps,
+    a 43 GB state cache) in the benchmark's launch configuration: seeded
+    samples of 4 rows per partition on two heads against the oracle, plus the
+    whole hit/age/store bookkeeping, which must be bit-exact."""
+    s = W.spec("video_long")
+    steps = [(q, k, v) for _, q, k, v in W.video_trajectory(s, device="cuda")]
+    plans = [W.plan_for_step(s, t).numpy() for t in range(s.steps)]
+    _run_steps(api, s, steps, plans, rows=W.sample_rows(s, 4).numpy(), heads=[0, 39])
+    del steps
+    torch.cuda.empty_cache()
+
+
 def test_step_f32_with_reuse(api):
     s = W.spec("tiny_f32", P=8)
     q, k, v = (x.cuda() for x in W.iid_qkv(s))
