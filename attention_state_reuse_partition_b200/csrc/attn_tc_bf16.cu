@@ -67,8 +67,9 @@ struct Layout {
 
 struct Ctrl {
   uint64_t q_full;
-  uint64_t k_full[NST], k_empty[NST];
-  uint64_t v_full[NST], v_empty[NST];
+  // load unit u carries K_u and V_{u-1} (K stage u % 2, V stage (u-1) % 2):
+  // exactly what the burst of tile u-1 needs
+  uint64_t kv_full[NST], kv_empty[NST];
   uint64_t s_full[NQ], p_full[NQ], o_ready[NQ], o_free[NQ];
   uint64_t drain;
   uint32_t tmem_base;
@@ -178,10 +179,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(&c.q_full, 1);
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&c.k_full[s], 1);
-      mbar_init(&c.k_empty[s], 1);
-      mbar_init(&c.v_full[s], 1);
-      mbar_init(&c.v_empty[s], 1);
+      mbar_init(&c.kv_full[s], 1);
+      mbar_init(&c.kv_empty[s], 1);
     }
     for (int t = 0; t < NQ; ++t) {
       mbar_init(&c.s_full[t], 1);
@@ -218,29 +217,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int rg = 0; rg < Lay::NREG; ++rg)
           tma_load_3d(smem + Lay::Q_OFF + t * Lay::TILE_BYTES + rg * REGION, &tm_q, &c.q_full, rg * 64,
                       q_lo + t * BM, bh);
+      // units 0..n_tiles: K_u (u < n_tiles) and V_{u-1} (u >= 1)
       TileWalk w;
-      int j = 0;
-      for (w.start(&c.sched); w.valid(); w.next(), ++j) {
-        const int st = j % NST;
-        const uint32_t ph = (j / NST) & 1;
-        if (!mbar_wait(&c.k_empty[st], ph ^ 1, abort_flag, budget)) break;
-        uint8_t* sK = smem + Lay::K_OFF + st * Lay::TILE_BYTES;
-        mbar_arrive_expect_tx(&c.k_full[st], Lay::TILE_BYTES);
-        for (int rg = 0; rg < Lay::NREG; ++rg)
-          tma_load_3d(sK + rg * REGION, &tm_k, &c.k_full[st], rg * 64, w.t, bh);
-        if (!mbar_wait(&c.v_empty[st], ph ^ 1, abort_flag, budget)) { ++j; break; }
-        uint8_t* sV = smem + Lay::V_OFF + st * Lay::TILE_BYTES;
-        mbar_arrive_expect_tx(&c.v_full[st], Lay::TILE_BYTES);
-        for (int rg = 0; rg < Lay::NREG; ++rg)
-          tma_load_3d(sV + rg * REGION, &tm_v, &c.v_full[st], rg * 64, w.t, bh);
+      w.start(&c.sched);
+      int prev_t = 0;  // KV row of tile u-1
+      int u = 0;
+      for (; u <= n_tiles; ++u) {
+        const int slot = u % NST;
+        if (!mbar_wait(&c.kv_empty[slot], ((u / NST) & 1) ^ 1, abort_flag, budget)) break;
+        const bool has_k = u < n_tiles, has_v = u >= 1;
+        mbar_arrive_expect_tx(&c.kv_full[slot], (has_k ? Lay::TILE_BYTES : 0) + (has_v ? Lay::TILE_BYTES : 0));
+        if (has_v) {
+          uint8_t* sV = smem + Lay::V_OFF + ((u - 1) % NST) * Lay::TILE_BYTES;
+          for (int rg = 0; rg < Lay::NREG; ++rg)
+            tma_load_3d(sV + rg * REGION, &tm_v, &c.kv_full[slot], rg * 64, prev_t, bh);
+        }
+        if (has_k) {
+          uint8_t* sK = smem + Lay::K_OFF + (u % NST) * Lay::TILE_BYTES;
+          for (int rg = 0; rg < Lay::NREG; ++rg)
+            tma_load_3d(sK + rg * REGION, &tm_k, &c.kv_full[slot], rg * 64, w.t, bh);
+          prev_t = w.t;
+          w.next();
+        }
       }
       // before the CTA may exit, every issued load must have landed
       if (*abort_flag) {
         drain_wait(&c.q_full, 0, budget);
-        for (int jj = max(0, j - NST); jj < j; ++jj) {
-          drain_wait(&c.k_full[jj % NST], (jj / NST) & 1, budget);
-          drain_wait(&c.v_full[jj % NST], (jj / NST) & 1, budget);
-        }
+        for (int uu = max(0, u - NST); uu < u; ++uu) drain_wait(&c.kv_full[uu % NST], (uu / NST) & 1, budget);
       }
     }
   } else if (warp == 1) {
@@ -270,30 +273,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           umma_bf16_ts(tmem + Lay::O_COL + t * D, tmem + t * BN + kk * 8, dv + ((kk * 16 * 128) >> 4),
                        IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
       };
-      bool ok = mbar_wait(&c.q_full, 0, abort_flag, budget) && mbar_wait(&c.k_full[0], 0, abort_flag, budget);
+      // unit 0 (K_0) for the first QKs, unit 1 (V_0, K_1) for the first burst
+      bool ok = mbar_wait(&c.q_full, 0, abort_flag, budget) && mbar_wait(&c.kv_full[0], 0, abort_flag, budget);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < NQ; ++t) {
           issue_qk(t, 0);
           umma_commit(&c.s_full[t]);
         }
-        umma_commit(&c.k_empty[0]);
+        umma_commit(&c.kv_empty[0]);
+        ok = mbar_wait(&c.kv_full[1 % NST], (1 / NST) & 1, abort_flag, budget);
         TileWalk w;
         int j = 0, group = 0;
         for (w.start(&c.sched); w.valid() && ok; w.next(), ++j) {
           const bool first = w.first(), last = w.last();
           if (first && j > 0) ++group;
           const bool has_next = j + 1 < n_tiles;
-          const int st = j % NST;
           for (int t = 0; t < NQ; ++t) {
-            // every wait of the burst first (the data waits, satisfied early,
-            // before the softmax handshake), then the 16 MMAs back to back
-            if (t == 0 && !mbar_wait(&c.v_full[st], (j / NST) & 1, abort_flag, budget)) ok = false;
-            if (ok && t == 0 && has_next &&
-                !mbar_wait(&c.k_full[(j + 1) % NST], ((j + 1) / NST) & 1, abort_flag, budget))
-              ok = false;
-            if (ok && first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget))
-              ok = false;
+            // the burst's data (unit j+1) was waited for earlier; here only
+            // the softmax handshake, then the 16 MMAs back to back
+            if (first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget)) ok = false;
             if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag, budget)) ok = false;
             if (!ok) break;
             tc_fence_after();
@@ -302,8 +301,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (last) umma_commit(&c.o_ready[t]);
             if (has_next) umma_commit(&c.s_full[t]);
             if (t == NQ - 1) {
-              umma_commit(&c.v_empty[st]);
-              if (has_next) umma_commit(&c.k_empty[(j + 1) % NST]);
+              umma_commit(&c.kv_empty[(j + 1) % NST]);  // unit j+1: V_j and K_{j+1} consumed
+            } else if (has_next) {
+              // data of the next burst, waited for while the other tile's softmax runs
+              const int u = j + 2;
+              if (!mbar_wait(&c.kv_full[u % NST], (u / NST) & 1, abort_flag, budget)) {
+                ok = false;
+                break;
+              }
             }
           }
         }
