@@ -240,3 +240,134 @@ def mse(a, b):
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     return float(np.mean((a - b) ** 2))
+
+
+# ---------------------------------------------------------------------------
+# the anchor-guided planner (DiTango review: Referee Report major comments
+# 1-3 and the Axiom & Free-Parameter Ledger; Eq. 7-10, 12, 13, Algorithm 1)
+# ---------------------------------------------------------------------------
+# Readings (the page names the quantities but prints few formulas):
+# * the importance of KV partition j for query partition i is the softmax of
+#   the partitions' LSEs, w(i,j) = mean over the rows r of i (and over b, h)
+#   of exp(LSE_ij[r] - LSE_i[r]), taken at an anchor (Eq. 8); sum_j w = 1;
+# * the scale ratio is alpha(i,j) = ||OUT_ij||_F / ||OUT_ii||_F at the anchor,
+#   the Frobenius norms running over the rows of i, b, h and d (Eq. 9);
+# * the local drift is D(i,t) = ||OUT_t(i,i) - OUT_ta(i,i)||_F against the
+#   anchor's local state, and delta(i,j,t) = alpha(i,j) * D(i,t) (Eq. 10);
+# * ASE(i,j,t) = w(i,j) * delta(i,j,t) (Eq. 7; groups of one pair, Eq. 12);
+# * selection (Eq. 13 with the adaptive threshold of Algorithm 1): pairs with
+#   |i-j| <= window are always fresh; of the remaining pairs, the
+#   floor(R * count) with the smallest ASE are reused (threshold = that
+#   order statistic), ties broken by (i, j); the others are fresh and refresh
+#   their cache entry;
+# * an anchor is taken when no anchor exists or when the relative local drift
+#   max_i D(i,t) / ||OUT_ta(i,i)||_F exceeds eps_local; at an anchor every pair
+#   is fresh and every remote pair is stored.
+
+def anchor_weights(lse_pairs, lse_full):
+    """w(i, j) for one query partition i: lse_pairs [P, ...rows] holds LSE_ij
+    for every j, lse_full [...rows] the LSE of the composition."""
+    lse_pairs = np.asarray(lse_pairs, dtype=np.float64)
+    lse_full = np.asarray(lse_full, dtype=np.float64)
+    return np.exp(lse_pairs - lse_full[None]).reshape(lse_pairs.shape[0], -1).mean(axis=1)
+
+
+def frob(x):
+    return float(np.sqrt(np.sum(np.asarray(x, dtype=np.float64) ** 2)))
+
+
+def scale_ratios(out_pairs, i):
+    """alpha(i, j) = ||OUT_ij|| / ||OUT_ii|| for one query partition i;
+    out_pairs [P, ...rows, d]."""
+    norms = np.array([frob(o) for o in out_pairs])
+    return norms / norms[i]
+
+
+def local_drift(out_now, out_anchor):
+    """(||OUT_t - OUT_ta||_F, ||OUT_ta||_F) of one query partition's local state."""
+    return frob(np.asarray(out_now, dtype=np.float64) - np.asarray(out_anchor, dtype=np.float64)), frob(out_anchor)
+
+
+def ase(w, alpha, drift):
+    """ASE(i, j) = w(i, j) * alpha(i, j) * D(i): w, alpha [P, P], drift [P]."""
+    return np.asarray(w, dtype=np.float64) * np.asarray(alpha, dtype=np.float64) * \
+        np.asarray(drift, dtype=np.float64)[:, None]
+
+
+def select_plan(ase_ij, window, reuse_ratio):
+    """Plan codes from ASE values (see the readings above)."""
+    ase_ij = np.asarray(ase_ij, dtype=np.float64)
+    P = ase_ij.shape[0]
+    plan = np.full((P, P), PLAN_FRESH_STORE, dtype=np.uint8)
+    remote = []
+    for i in range(P):
+        for j in range(P):
+            if abs(i - j) <= window:
+                plan[i, j] = PLAN_FRESH
+            else:
+                remote.append((ase_ij[i, j], i, j))
+    remote.sort()
+    n_reuse = int(np.floor(reuse_ratio * len(remote) + 1e-9))
+    for _, i, j in remote[:n_reuse]:
+        plan[i, j] = PLAN_REUSE
+    return plan
+
+
+def anchor_plan(P, window):
+    """Every pair fresh; every pair outside the window stored."""
+    i = np.arange(P)[:, None]
+    j = np.arange(P)[None, :]
+    return np.where(np.abs(i - j) <= window, PLAN_FRESH, PLAN_FRESH_STORE).astype(np.uint8)
+
+
+class Planner:
+    """The planner's state between steps: the anchor's w, alpha and local
+    states (OUT_ta(i,i) for every i, [B,H,S,d])."""
+
+    def __init__(self, P, window, reuse_ratio, eps_local):
+        self.P, self.window = P, window
+        self.reuse_ratio, self.eps_local = reuse_ratio, eps_local
+        self.has_anchor = False
+        self.w = np.zeros((P, P))
+        self.alpha = np.zeros((P, P))
+        self.local_anchor = None
+
+
+def planner_next(pl, local_now, n):
+    """Plan of the next step from the current local states (OUT_t(i,i) for
+    every i, [B,H,S,d] with partition i at rows [i n, (i+1) n)).  Returns
+    (plan, is_anchor, drift [P], ase [P,P] or None)."""
+    P = pl.P
+    if not pl.has_anchor:
+        pl.local_anchor = np.array(local_now, dtype=np.float64, copy=True)
+        return anchor_plan(P, pl.window), True, np.zeros(P), None
+    drift = np.zeros(P)
+    rel = np.zeros(P)
+    for i in range(P):
+        dd, nrm = local_drift(local_now[..., i * n:(i + 1) * n, :], pl.local_anchor[..., i * n:(i + 1) * n, :])
+        drift[i] = dd
+        rel[i] = dd / nrm if nrm > 0 else 0.0
+    if rel.max() > pl.eps_local:
+        pl.local_anchor = np.array(local_now, dtype=np.float64, copy=True)
+        return anchor_plan(P, pl.window), True, drift, None
+    a = ase(pl.w, pl.alpha, drift)
+    return select_plan(a, pl.window, pl.reuse_ratio), False, drift, a
+
+
+def planner_commit_anchor(pl, cache, lse_full, rows_of, n):
+    """After an anchor step: w and alpha of every stored pair from the cache
+    entries, the composed LSE and the anchor's local states.  ``rows_of(i)``
+    gives the positions, within the evaluated rows, of partition i's rows
+    (the same rows the cache entries hold)."""
+    P = pl.P
+    for i in range(P):
+        sel = rows_of(i)
+        local = pl.local_anchor[..., i * n:(i + 1) * n, :]
+        local_norm = frob(local)
+        for j in range(P):
+            if (i, j) not in cache.entry or cache.t_c[i, j] < 0 or abs(i - j) <= pl.window:
+                continue
+            o, l = cache.entry[(i, j)]
+            pl.w[i, j] = float(np.mean(np.exp(np.asarray(l) - np.asarray(lse_full)[..., sel])))
+            pl.alpha[i, j] = frob(o) / local_norm
+    pl.has_anchor = True

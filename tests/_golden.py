@@ -31,3 +31,18 @@ def load_plan_fixture(name="plan_4x4.txt"):
             case["age"] = _matrix(lines, P, np.int32)
         cases.append(case)
     return P, cases
+
+
+def load_select_fixture(name="select_4x4.txt"):
+    """Returns (P, window, ase [P,P] float64, [(ratio, plan [P,P] uint8)])."""
+    with open(os.path.join(GOLDEN, name)) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.lstrip().startswith("#")]
+    P = int(lines.pop(0).split()[1])
+    window = int(lines.pop(0).split()[1])
+    assert lines.pop(0) == "ase"
+    ase = np.array([[float(x) for x in lines.pop(0).split()] for _ in range(P)])
+    cases = []
+    while lines:
+        ratio = float(lines.pop(0).split()[1])
+        cases.append((ratio, _matrix(lines, P, np.uint8)))
+    return P, window, ase, cases

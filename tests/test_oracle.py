@@ -27,7 +27,7 @@ import scipy.special
 import torch
 
 from oracle import as_oracle
-from tests._golden import load_plan_fixture
+from tests._golden import load_plan_fixture, load_select_fixture
 
 TOL = 1e-11
 
@@ -263,9 +263,98 @@ def pin_step_reuse_mixed(o):
     assert cache.t_c[0, 4] == 1 and cache.t_c[0, 3] == 0
 
 
+# ---------------------------------------------------------------------------
+# planner pins (DiTango review: Eq. 7-10, 12, 13 and Algorithm 1 as read in
+# the oracle's planner section)
+# ---------------------------------------------------------------------------
+
+def pin_planner_weights(o):
+    r = _rng(20)
+    q, k, v = (r.normal(size=(1, 2, 24, 8)) for _ in range(3))
+    states = o.partition_states(q, k, v, 0.4, 4)
+    _, full_l = o.full_attention(q, k, v, 0.4)
+    w = o.anchor_weights(np.stack([l for _, l in states]), full_l)
+    _close(w.sum(), 1.0, 1e-12, "weights sum to 1")       # softmax over partitions
+    assert np.all(w > 0)
+    w_eq = o.anchor_weights(np.zeros((5, 7)), np.full(7, math.log(5)))
+    _close(w_eq, np.full(5, 0.2), 1e-12, "equal LSEs: uniform weights")
+    a, b = 0.3, -1.1
+    lse2 = np.array([[a] * 3, [b] * 3])
+    w2 = o.anchor_weights(lse2, np.full(3, math.log(math.exp(a) + math.exp(b))))
+    _close(w2, np.array([math.exp(a), math.exp(b)]) / (math.exp(a) + math.exp(b)), 1e-12, "two-partition weights")
+
+
+def pin_planner_ratios(o):
+    r = _rng(21)
+    base = r.normal(size=(2, 6, 4))
+    outs = np.stack([base, 3.0 * base, -0.5 * base, np.zeros_like(base)])
+    al = o.scale_ratios(outs, 0)
+    _close(al, np.array([1.0, 3.0, 0.5, 0.0]), 1e-12, "scale ratios")
+    _close(o.scale_ratios(outs, 1)[1], 1.0, 1e-12, "local ratio is 1")
+
+
+def pin_planner_drift(o):
+    r = _rng(22)
+    anchor = r.normal(size=(2, 5, 4))
+    d0, n0 = o.local_drift(anchor, anchor)
+    assert d0 == 0.0
+    _close(n0, math.sqrt(float(np.sum(anchor ** 2))), 1e-12, "anchor norm")
+    d1, _ = o.local_drift(anchor + 0.25, anchor)
+    _close(d1, 0.25 * math.sqrt(anchor.size), 1e-12, "drift of a constant shift")
+
+
+def pin_planner_select(o):
+    P, window, a, cases = load_select_fixture()
+    for ratio, plan in cases:
+        assert np.array_equal(o.select_plan(a, window, ratio), plan), f"selection at R={ratio}"
+    assert (o.select_plan(a, P, 0.7) == o_FRESH).all(), "window covering everything: all fresh"
+    # ASE = w * alpha * drift (Eq. 7 with Eq. 10): with w = 1/2 everywhere,
+    # alpha decides the order; by hand the smallest remote ASE is (0, 1)
+    w = np.full((2, 2), 0.5)
+    alpha = np.array([[1.0, 0.2], [4.0, 1.0]])
+    aa = o.ase(w, alpha, np.array([1.0, 0.5]))
+    _close(aa, np.array([[0.5, 0.1], [1.0, 0.25]]), 1e-12, "ASE worked example")
+    assert np.array_equal(o.select_plan(aa, 0, 0.5), np.array([[1, 0], [2, 1]], np.uint8))
+
+
+def pin_planner_trajectory(o):
+    """Inputs that do not move: the first step is an anchor, the next one
+    reuses exactly floor(R * #remote) pairs (all ASE are 0) and still equals
+    full attention; a large change triggers a new anchor."""
+    r = _rng(23)
+    B, H, S, d, P = 1, 1, 32, 4, 4
+    n = S // P
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    pl = o.Planner(P, window=0, reuse_ratio=0.5, eps_local=0.05)
+    cache = o.StateCache(P)
+    rows = np.arange(S)
+    local = np.concatenate([o.attention_state(q[..., i * n:(i + 1) * n, :], k[..., i * n:(i + 1) * n, :],
+                                              v[..., i * n:(i + 1) * n, :], 0.5)[0] for i in range(P)], axis=-2)
+    plan0, anchor0, _, _ = o.planner_next(pl, local, n)
+    assert anchor0 and np.array_equal(plan0, o.anchor_plan(P, 0))
+    _, lse0, _, _ = o.step(cache, q, k, v, plan0, 0, 0.5)
+    o.planner_commit_anchor(pl, cache, lse0, lambda i: np.arange(i * n, (i + 1) * n), n)
+    # the stored (remote) weights plus the local partition's weight sum to 1
+    w_loc = np.array([float(np.mean(np.exp(o.attention_state(
+        q[..., i * n:(i + 1) * n, :], k[..., i * n:(i + 1) * n, :], v[..., i * n:(i + 1) * n, :], 0.5)[1]
+        - lse0[..., i * n:(i + 1) * n]))) for i in range(P)])
+    _close(pl.w.sum(axis=1) + w_loc, np.ones(P), 1e-12, "anchor weights of a query partition")
+    plan1, anchor1, drift1, a1 = o.planner_next(pl, local, n)
+    assert not anchor1 and np.all(drift1 == 0) and np.all(a1 == 0)
+    assert int((plan1 == o_REUSE).sum()) == (P * P - P) // 2
+    out1, _, _, _ = o.step(cache, q, k, v, plan1, 1, 0.5)
+    _close(out1, _sdpa(q, k, v, 0.5), TOL, "reuse of unchanged states")
+    k2 = r.normal(size=k.shape)
+    local2 = np.concatenate([o.attention_state(q[..., i * n:(i + 1) * n, :], k2[..., i * n:(i + 1) * n, :],
+                                               v[..., i * n:(i + 1) * n, :], 0.5)[0] for i in range(P)], axis=-2)
+    _, anchor2, _, _ = o.planner_next(pl, local2, n)
+    assert anchor2, "a large local drift must trigger an anchor"
+
+
 PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_forms,
         pin_compose_closed, pin_assoc_comm, pin_split_invariance, pin_single_partition,
-        pin_plan_golden, pin_step_all_fresh, pin_step_reuse_identical, pin_step_reuse_mixed]
+        pin_plan_golden, pin_step_all_fresh, pin_step_reuse_identical, pin_step_reuse_mixed,
+        pin_planner_weights, pin_planner_ratios, pin_planner_drift, pin_planner_select, pin_planner_trajectory]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -278,7 +367,8 @@ def test_oracle_passes_pin(pin):
 # ---------------------------------------------------------------------------
 
 _orig = {name: getattr(as_oracle, name) for name in
-         ("attention_state", "compose", "compose_pair", "resolve_plan", "step", "partition_bounds")}
+         ("attention_state", "compose", "compose_pair", "resolve_plan", "step", "partition_bounds",
+          "anchor_weights", "scale_ratios", "local_drift", "select_plan", "ase")}
 
 
 def _m_no_normalise(q, k, v, scale):
@@ -352,6 +442,34 @@ def _m_bounds_shift(S, P):
     return b[1:] + b[:1]
 
 
+def _m_weights_unnormalised(lse_pairs, lse_full):
+    lse_pairs = np.asarray(lse_pairs, dtype=np.float64)
+    return np.exp(lse_pairs).reshape(lse_pairs.shape[0], -1).mean(axis=1)
+
+
+def _m_ratios_inverted(out_pairs, i):
+    r = _orig["scale_ratios"](out_pairs, i)
+    with np.errstate(divide="ignore"):
+        return np.where(r > 0, 1.0 / r, 0.0)
+
+
+def _m_drift_relative(out_now, out_anchor):
+    d, nrm = _orig["local_drift"](out_now, out_anchor)
+    return (d / nrm if nrm > 0 else 0.0), nrm
+
+
+def _m_select_largest(ase_ij, window, reuse_ratio):
+    return _orig["select_plan"](-np.asarray(ase_ij), window, reuse_ratio)
+
+
+def _m_select_window(ase_ij, window, reuse_ratio):
+    return _orig["select_plan"](ase_ij, window - 1, reuse_ratio)
+
+
+def _m_ase_no_alpha(w, alpha, drift):
+    return _orig["ase"](w, np.ones_like(np.asarray(alpha, dtype=np.float64)), drift)
+
+
 MUTANTS = {
     "attention_state: OUT not normalised": ("attention_state", _m_no_normalise),
     "attention_state: LSE without the scale": ("attention_state", _m_lse_unscaled),
@@ -365,6 +483,12 @@ MUTANTS = {
     "resolve_plan: hit on fresh": ("resolve_plan", _m_hit_fresh),
     "step: stores plain-fresh pairs": ("step", _m_store_all_fresh),
     "partition_bounds: off by one partition": ("partition_bounds", _m_bounds_shift),
+    "anchor_weights: not normalised by the composed LSE": ("anchor_weights", _m_weights_unnormalised),
+    "scale_ratios: inverted": ("scale_ratios", _m_ratios_inverted),
+    "local_drift: relative instead of absolute": ("local_drift", _m_drift_relative),
+    "select_plan: reuses the largest ASE": ("select_plan", _m_select_largest),
+    "select_plan: window off by one": ("select_plan", _m_select_window),
+    "ase: drops the scale ratio": ("ase", _m_ase_no_alpha),
 }
 
 
