@@ -22,7 +22,8 @@ STATUS_NAMES = {
 # every entry point declared in include/as_partition.h
 EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as_cache_bytes",
            "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe",
-           "as_debug_exp2")
+           "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
+           "as_plan_select", "as_planner_next", "as_planner_commit_anchor")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -33,6 +34,19 @@ class AsCacheStruct(ctypes.Structure):
         ("out_planes", ctypes.c_void_p),
         ("lse_planes", ctypes.c_void_p),
         ("t_c", ctypes.c_int32 * (AS_MAX_P * AS_MAX_P)),
+    ]
+
+
+class AsPlannerStruct(ctypes.Structure):
+    _fields_ = [
+        ("magic", ctypes.c_uint32),
+        ("P", ctypes.c_int), ("window", ctypes.c_int),
+        ("reuse_ratio", ctypes.c_double), ("eps_local", ctypes.c_double),
+        ("has_anchor", ctypes.c_int),
+        ("w", ctypes.c_double * (AS_MAX_P * AS_MAX_P)),
+        ("alpha", ctypes.c_double * (AS_MAX_P * AS_MAX_P)),
+        ("drift", ctypes.c_double * AS_MAX_P),
+        ("rel_drift", ctypes.c_double * AS_MAX_P),
     ]
 
 
@@ -71,6 +85,23 @@ def _load() -> ctypes.CDLL:
     lib.as_device_status.argtypes = [vp, ctypes.POINTER(u32)]
     lib.as_debug_timeout_probe.restype = c_int
     lib.as_debug_timeout_probe.argtypes = [u32, vp]
+    dbl = ctypes.c_double
+    lib.as_planner_init.restype = c_int
+    lib.as_planner_init.argtypes = [ctypes.POINTER(AsPlannerStruct), c_int, c_int, dbl, dbl]
+    lib.as_planner_scratch_bytes.restype = sz
+    lib.as_planner_scratch_bytes.argtypes = [c_int, c_int, c_int]
+    lib.as_local_states.restype = c_int
+    lib.as_local_states.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, ctypes.c_float, vp, vp, vp]
+    lib.as_plan_drift.restype = c_int
+    lib.as_plan_drift.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, vp, sz, vp, vp, vp]
+    lib.as_plan_select.restype = c_int
+    lib.as_plan_select.argtypes = [vp, c_int, c_int, dbl, vp]
+    lib.as_planner_next.restype = c_int
+    lib.as_planner_next.argtypes = [ctypes.POINTER(AsPlannerStruct), vp, vp, c_int, c_int, c_int, c_int, vp, sz, vp,
+                                    ctypes.POINTER(c_int), vp, vp]
+    lib.as_planner_commit_anchor.restype = c_int
+    lib.as_planner_commit_anchor.argtypes = [ctypes.POINTER(AsPlannerStruct), ctypes.POINTER(AsCacheStruct), vp, vp,
+                                             vp, vp, sz, vp]
     lib.as_debug_exp2.restype = c_int
     lib.as_debug_exp2.argtypes = [vp, vp, i64, c_int, vp]
     return lib

@@ -12,11 +12,13 @@ import torch
 
 from . import _lib
 from ._lib import (AS_BF16, AS_F32, AS_PLAN_FRESH, AS_PLAN_FRESH_STORE, AS_PLAN_REUSE, AsCacheStruct,
-                   AsError, LIB, check)
+                   AsError, AsPlannerStruct, LIB, check)
 
 __all__ = ["as_partition_attn", "as_compose", "as_cache_bytes", "as_cache_init", "as_plan_resolve", "as_step",
            "as_device_status", "as_debug_timeout_probe", "as_version", "AsCache", "AsError",
-           "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE"]
+           "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE", "AsPlanner", "as_planner_init",
+           "as_planner_scratch_bytes", "as_local_states", "as_plan_drift", "as_plan_select", "as_planner_next",
+           "as_planner_commit_anchor"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -162,6 +164,111 @@ def as_step(cache: AsCache, q, k, v, plan, step: int, scale: Optional[float] = N
                       float(scale), arr.ctypes.data, int(step), _dev(out, "out"), _dev(lse, "lse"),
                       hit.ctypes.data, age.ctypes.data, _stream_ptr(stream)))
     return out, lse, hit.reshape(P, P), age.reshape(P, P)
+
+
+# ---------------------------------------------------------------------------
+# the anchor-guided planner
+# ---------------------------------------------------------------------------
+
+def as_planner_scratch_bytes(B: int, H: int, P: int) -> int:
+    return int(LIB.as_planner_scratch_bytes(B, H, P))
+
+
+class AsPlanner:
+    """The planner's C struct plus its device buffers (scratch and the anchor's
+    local states), allocated with torch."""
+
+    def __init__(self, P: int, window: int, reuse_ratio: float, eps_local: float, B: int = 0, H: int = 0,
+                 S: int = 0, d: int = 0, device="cuda"):
+        self.struct = AsPlannerStruct()
+        check(LIB.as_planner_init(ctypes.byref(self.struct), P, window, float(reuse_ratio), float(eps_local)))
+        self.P = P
+        self.scratch = None
+        self.local_anchor = None
+        if B:
+            nbytes = as_planner_scratch_bytes(B, H, P)
+            self.scratch = torch.empty(nbytes // 8 + 1, dtype=torch.float64, device=device)
+            self.local_anchor = torch.zeros((B, H, S, d), dtype=torch.float32, device=device)
+
+    def _arr(self, name, n):
+        return np.ctypeslib.as_array(getattr(self.struct, name))[:n].copy()
+
+    @property
+    def has_anchor(self) -> bool:
+        return bool(self.struct.has_anchor)
+
+    @property
+    def w(self):
+        return self._arr("w", self.P * self.P).reshape(self.P, self.P)
+
+    @property
+    def alpha(self):
+        return self._arr("alpha", self.P * self.P).reshape(self.P, self.P)
+
+    @property
+    def drift(self):
+        return self._arr("drift", self.P)
+
+    @property
+    def rel_drift(self):
+        return self._arr("rel_drift", self.P)
+
+
+def as_planner_init(P, window, reuse_ratio, eps_local, B=0, H=0, S=0, d=0, device="cuda") -> AsPlanner:
+    return AsPlanner(P, window, reuse_ratio, eps_local, B, H, S, d, device)
+
+
+def as_local_states(q, k, v, P: int, scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """Local states AS(i, i) of every query partition: out [B,H,S,d], lse [B,H,S]."""
+    B, H, S, d = q.shape
+    scale = 1.0 / d ** 0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, S, d), device=q.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    check(LIB.as_local_states(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q), B, H, S, d, P,
+                              float(scale), _dev(out, "out"), _dev(lse, "lse"), _stream_ptr(stream)))
+    return out, lse
+
+
+def as_plan_drift(now, anchor, P: int, scratch, stream=None):
+    """(drift [P], norm [P]) of every partition's local state against the anchor's."""
+    B, H, S, d = now.shape
+    drift = np.zeros(P, dtype=np.float64)
+    norm = np.zeros(P, dtype=np.float64)
+    check(LIB.as_plan_drift(_dev(now, "now"), _dev(anchor, "anchor"), B, H, S, d, P, _dev(scratch, "scratch"),
+                            scratch.numel() * scratch.element_size(), drift.ctypes.data, norm.ctypes.data,
+                            _stream_ptr(stream)))
+    return drift, norm
+
+
+def as_plan_select(ase, window: int, reuse_ratio: float):
+    """Host-only plan selection from ASE values [P, P]."""
+    a = np.ascontiguousarray(np.asarray(ase, dtype=np.float64))
+    P = a.shape[0]
+    plan = np.zeros(P * P, dtype=np.uint8)
+    check(LIB.as_plan_select(a.ctypes.data, P, int(window), float(reuse_ratio), plan.ctypes.data))
+    return plan.reshape(P, P)
+
+
+def as_planner_next(pl: AsPlanner, local_now, stream=None):
+    """(plan [P,P], is_anchor, ase [P,P]) of the next step."""
+    B, H, S, d = local_now.shape
+    P = pl.P
+    plan = np.zeros(P * P, dtype=np.uint8)
+    ase = np.zeros(P * P, dtype=np.float64)
+    is_anchor = ctypes.c_int(0)
+    check(LIB.as_planner_next(ctypes.byref(pl.struct), _dev(local_now, "local_now"), _dev(pl.local_anchor, "anchor"),
+                              B, H, S, d, _dev(pl.scratch, "scratch"), pl.scratch.numel() * 8, plan.ctypes.data,
+                              ctypes.byref(is_anchor), ase.ctypes.data, _stream_ptr(stream)))
+    return plan.reshape(P, P), bool(is_anchor.value), ase.reshape(P, P)
+
+
+def as_planner_commit_anchor(pl: AsPlanner, cache: AsCache, lse_full, plan, stream=None):
+    arr = _plan_bytes(plan, pl.P)
+    check(LIB.as_planner_commit_anchor(ctypes.byref(pl.struct), ctypes.byref(cache.struct), _dev(lse_full, "lse"),
+                                       _dev(pl.local_anchor, "anchor"), arr.ctypes.data, _dev(pl.scratch, "scratch"),
+                                       pl.scratch.numel() * 8, _stream_ptr(stream)))
 
 
 def as_device_status(stream=None) -> int:

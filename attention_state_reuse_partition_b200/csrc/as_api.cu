@@ -5,17 +5,22 @@
 // Semantics follow DiTango (arXiv 2607.15650; review page: "What carries the
 // argument" for the attention state, Axiom & Free-Parameter Ledger Eq. 1-2 for
 // composition, Core claim and Referee Report "Summary" for fresh/reuse steps).
+#include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <tuple>
+#include <vector>
 
 #include "as_kernels.h"
 #include "as_partition.h"
 
 namespace {
 
-constexpr uint32_t CACHE_MAGIC = 0x41535043u;  // "ASPC"
+constexpr uint32_t CACHE_MAGIC = 0x41535043u;    // "ASPC"
+constexpr uint32_t PLANNER_MAGIC = 0x41535050u;  // "ASPP"
 thread_local std::string g_err;
 
 as_status fail(as_status s, const char* fmt, ...) {
@@ -99,6 +104,62 @@ as_status resolve(const as_cache* c, const uint8_t* plan, int step, uint8_t* hit
     if (hit) hit[x] = r ? 1 : 0;
     if (age) age[x] = r ? step - c->t_c[x] : 0;
   }
+  return AS_OK;
+}
+
+// planner scratch: partials [P*P][BH][2] doubles, then sums [P*P][2] doubles
+size_t planner_scratch(int B, int H, int P) {
+  return (static_cast<size_t>(P) * P * B * H * 2 + static_cast<size_t>(P) * P * 2) * sizeof(double);
+}
+
+as_status check_scratch(void* scratch, size_t bytes, int B, int H, int P) {
+  if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 7u) != 0)
+    return fail(AS_ERR_INVALID_ARG, "planner scratch must be non-null and 8-byte aligned");
+  if (bytes < planner_scratch(B, H, P))
+    return fail(AS_ERR_INVALID_ARG, "planner scratch has %zu bytes, needs %zu", bytes, planner_scratch(B, H, P));
+  return AS_OK;
+}
+
+// selection from ASE values: |i-j| <= window fresh; of the rest the
+// floor(R * count) smallest (ties by (i, j)) reused, the others fresh + stored
+void select_plan(const double* ase, int P, int window, double ratio, uint8_t* plan) {
+  std::vector<std::tuple<double, int, int>> remote;
+  for (int i = 0; i < P; ++i)
+    for (int j = 0; j < P; ++j) {
+      if (std::abs(i - j) <= window) {
+        plan[i * P + j] = AS_PLAN_FRESH;
+      } else {
+        plan[i * P + j] = AS_PLAN_FRESH_STORE;
+        remote.emplace_back(ase[i * P + j], i, j);
+      }
+    }
+  std::sort(remote.begin(), remote.end());
+  const size_t n_reuse = static_cast<size_t>(std::floor(ratio * static_cast<double>(remote.size()) + 1e-9));
+  for (size_t x = 0; x < n_reuse && x < remote.size(); ++x)
+    plan[std::get<1>(remote[x]) * P + std::get<2>(remote[x])] = AS_PLAN_REUSE;
+}
+
+void anchor_plan(int P, int window, uint8_t* plan) {
+  for (int i = 0; i < P; ++i)
+    for (int j = 0; j < P; ++j) plan[i * P + j] = std::abs(i - j) <= window ? AS_PLAN_FRESH : AS_PLAN_FRESH_STORE;
+}
+
+// drift and anchor norms of every partition, host values
+as_status run_drift(const float* now, const float* anchor, int B, int H, int S, int d, int P, void* scratch,
+                    cudaStream_t st, double* h_sums /*[P][2]*/) {
+  double* partials = static_cast<double*>(scratch);
+  double* sums = partials + static_cast<size_t>(P) * P * B * H * 2;
+  cudaError_t e = asp::launch_drift(now, anchor, B * H, S, d, P, partials, sums, st);
+  if (e != cudaSuccess) return cuda_fail(e, "drift launch");
+  e = cudaMemcpyAsync(h_sums, sums, static_cast<size_t>(P) * 2 * sizeof(double), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "drift copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "drift sync");
+  return AS_OK;
+}
+
+as_status check_planner(const as_planner* pl) {
+  if (!pl || pl->magic != PLANNER_MAGIC) return fail(AS_ERR_INVALID_ARG, "planner not initialised by as_planner_init");
   return AS_OK;
 }
 
@@ -333,6 +394,166 @@ as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream) {
   if (s != AS_OK) return s;
   cudaError_t e = asp::launch_timeout_probe(poll_budget, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "timeout probe launch");
+  return ok();
+}
+
+as_status as_planner_init(as_planner* pl, int P, int window, double reuse_ratio, double eps_local) {
+  if (!pl) return fail(AS_ERR_INVALID_ARG, "null planner");
+  if (P < 1 || P > AS_MAX_P) return fail(AS_ERR_INVALID_ARG, "P must be in [1, %d]", AS_MAX_P);
+  if (window < 0) return fail(AS_ERR_INVALID_ARG, "window must be >= 0");
+  if (!(reuse_ratio >= 0.0 && reuse_ratio <= 1.0)) return fail(AS_ERR_INVALID_ARG, "reuse_ratio must be in [0, 1]");
+  if (!(eps_local >= 0.0)) return fail(AS_ERR_INVALID_ARG, "eps_local must be >= 0");
+  std::memset(pl, 0, sizeof(*pl));
+  pl->magic = PLANNER_MAGIC;
+  pl->P = P;
+  pl->window = window;
+  pl->reuse_ratio = reuse_ratio;
+  pl->eps_local = eps_local;
+  return ok();
+}
+
+size_t as_planner_scratch_bytes(int B, int H, int P) {
+  if (B < 1 || H < 1 || P < 1 || P > AS_MAX_P) return 0;
+  return planner_scratch(B, H, P);
+}
+
+as_status as_local_states(const void* q, const void* k, const void* v, as_dtype dt, int B, int H, int S, int d,
+                          int P, float scale, float* out, float* lse, void* stream) {
+  as_status s = check_shape(B, H, S, d, P);
+  if (s != AS_OK) return s;
+  if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+  if (!q || !k || !v || !out || !lse) return fail(AS_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(AS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (!(scale > 0.f)) return fail(AS_ERR_INVALID_ARG, "scale must be > 0");
+  asp::AttnLaunch L;
+  base_launch(L, q, k, v, B, H, S, d, P, scale);
+  L.n_blocks = P;
+  L.block_rows = S / P;
+  L.block_row0 = 0;
+  for (int i = 0; i < P; ++i) L.code[i * P + i] = AS_KCODE_EMIT;  // block i: its own partition only
+  L.out = out;
+  L.lse = lse;
+  L.out_rows = S;
+  L.out_row0 = 0;
+  L.dst_out = out;  // every emitted state goes to plane 0 at its own rows
+  L.dst_lse = lse;
+  L.dst_rows = S;
+  L.dst_row0 = 0;
+  if ((s = check_device()) != AS_OK) return s;
+  if ((s = launch_attn(L, dt, static_cast<cudaStream_t>(stream))) != AS_OK) return s;
+  return ok();
+}
+
+as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int S, int d, int P, void* scratch,
+                        size_t scratch_bytes, double* h_drift, double* h_norm, void* stream) {
+  as_status s = check_shape(B, H, S, d, P);
+  if (s != AS_OK) return s;
+  if (!now || !anchor || !h_drift || !h_norm) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
+  if ((s = check_device()) != AS_OK) return s;
+  std::vector<double> sums(static_cast<size_t>(P) * 2);
+  if ((s = run_drift(now, anchor, B, H, S, d, P, scratch, static_cast<cudaStream_t>(stream), sums.data())) != AS_OK)
+    return s;
+  for (int i = 0; i < P; ++i) {
+    h_drift[i] = std::sqrt(sums[i * 2 + 0]);
+    h_norm[i] = std::sqrt(sums[i * 2 + 1]);
+  }
+  return ok();
+}
+
+as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan) {
+  if (!h_ase || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if (P < 1 || P > AS_MAX_P || window < 0 || !(reuse_ratio >= 0.0 && reuse_ratio <= 1.0))
+    return fail(AS_ERR_INVALID_ARG, "bad P, window or reuse_ratio");
+  select_plan(h_ase, P, window, reuse_ratio, h_plan);
+  return ok();
+}
+
+as_status as_planner_next(as_planner* pl, const float* local_now, float* local_anchor, int B, int H, int S, int d,
+                          void* scratch, size_t scratch_bytes, uint8_t* h_plan, int* h_is_anchor, double* h_ase,
+                          void* stream) {
+  as_status s = check_planner(pl);
+  if (s != AS_OK) return s;
+  const int P = pl->P;
+  if ((s = check_shape(B, H, S, d, P)) != AS_OK) return s;
+  if (!local_now || !local_anchor || !h_plan || !h_is_anchor) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
+  if ((s = check_device()) != AS_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bool anchor = !pl->has_anchor;
+  for (int i = 0; i < P; ++i) pl->drift[i] = pl->rel_drift[i] = 0.0;
+  if (!anchor) {
+    std::vector<double> sums(static_cast<size_t>(P) * 2);
+    if ((s = run_drift(local_now, local_anchor, B, H, S, d, P, scratch, st, sums.data())) != AS_OK) return s;
+    double worst = 0.0;
+    for (int i = 0; i < P; ++i) {
+      pl->drift[i] = std::sqrt(sums[i * 2 + 0]);
+      const double nrm = std::sqrt(sums[i * 2 + 1]);
+      pl->rel_drift[i] = nrm > 0.0 ? pl->drift[i] / nrm : 0.0;
+      worst = std::max(worst, pl->rel_drift[i]);
+    }
+    anchor = worst > pl->eps_local;
+  }
+  if (h_ase) std::memset(h_ase, 0, static_cast<size_t>(P) * P * sizeof(double));
+  if (anchor) {
+    anchor_plan(P, pl->window, h_plan);
+    const size_t bytes = static_cast<size_t>(B) * H * S * d * sizeof(float);
+    cudaError_t e = cudaMemcpyAsync(local_anchor, local_now, bytes, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "anchor local-state copy");
+  } else {
+    std::vector<double> a(static_cast<size_t>(P) * P);
+    for (int i = 0; i < P; ++i)
+      for (int j = 0; j < P; ++j) a[i * P + j] = pl->w[i * P + j] * pl->alpha[i * P + j] * pl->drift[i];
+    select_plan(a.data(), P, pl->window, pl->reuse_ratio, h_plan);
+    if (h_ase) std::memcpy(h_ase, a.data(), a.size() * sizeof(double));
+  }
+  *h_is_anchor = anchor ? 1 : 0;
+  return ok();
+}
+
+as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const float* lse_full,
+                                   const float* local_anchor, const uint8_t* h_plan, void* scratch,
+                                   size_t scratch_bytes, void* stream) {
+  as_status s = check_planner(pl);
+  if (s != AS_OK) return s;
+  if ((s = check_cache(c)) != AS_OK) return s;
+  const int P = pl->P;
+  if (c->P != P) return fail(AS_ERR_INVALID_ARG, "cache and planner disagree on P");
+  if (!lse_full || !local_anchor || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  const int B = c->B, H = c->H, S = c->S, d = c->d, n = S / P;
+  if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
+  if ((s = check_device()) != AS_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  asp::PlanRows sel;
+  std::memset(&sel, 0, sizeof(sel));
+  for (int i = 0; i < P; ++i)
+    for (int j = 0; j < P; ++j)
+      sel.v[i * P + j] = (h_plan[i * P + j] == AS_PLAN_FRESH_STORE && std::abs(i - j) > pl->window) ? 1 : 0;
+  double* partials = static_cast<double*>(scratch);
+  double* sums = partials + static_cast<size_t>(P) * P * B * H * 2;
+  cudaError_t e = asp::launch_anchor_stats(c->out_planes, c->lse_planes, lse_full,
+                                           static_cast<long long>(B) * H * S * d, static_cast<long long>(B) * H * S,
+                                           P, B * H, S, d, sel, partials, sums, st);
+  if (e != cudaSuccess) return cuda_fail(e, "anchor statistics launch");
+  std::vector<double> stats(static_cast<size_t>(P) * P * 2);
+  e = cudaMemcpyAsync(stats.data(), sums, stats.size() * sizeof(double), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "anchor statistics copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "anchor statistics sync");
+  // norms of the anchor's local states (drift of the anchor against itself)
+  std::vector<double> norms(static_cast<size_t>(P) * 2);
+  if ((s = run_drift(local_anchor, local_anchor, B, H, S, d, P, scratch, st, norms.data())) != AS_OK) return s;
+  const double rows = static_cast<double>(B) * H * n;
+  for (int i = 0; i < P; ++i) {
+    const double local_norm = std::sqrt(norms[i * 2 + 1]);
+    for (int j = 0; j < P; ++j) {
+      if (!sel.v[i * P + j]) continue;
+      pl->w[i * P + j] = stats[(i * P + j) * 2 + 0] / rows;
+      pl->alpha[i * P + j] = local_norm > 0.0 ? std::sqrt(stats[(i * P + j) * 2 + 1]) / local_norm : 0.0;
+    }
+  }
+  pl->has_anchor = 1;
   return ok();
 }
 

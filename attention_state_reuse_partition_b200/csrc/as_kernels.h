@@ -66,7 +66,18 @@ struct ComposePlan {
   float* lse;
 };
 
+// pair selection for the planner's anchor statistics ([P][P], 1 = reduce)
+struct PlanRows {
+  uint8_t v[AS_MAX_P * AS_MAX_P];
+};
+
 cudaError_t launch_attn_tc_bf16(const AttnLaunch& L, cudaStream_t st);
+// planner reductions: partials scratch [K][BH][2] doubles, sums [K][2] doubles
+cudaError_t launch_drift(const float* now, const float* anchor, int BH, int S, int d, int P, double* partials,
+                         double* sums, cudaStream_t st);
+cudaError_t launch_anchor_stats(const float* cache_out, const float* cache_lse, const float* lse_full,
+                                long long plane_out, long long plane_lse, int P, int BH, int S, int d,
+                                const PlanRows& sel, double* partials, double* sums, cudaStream_t st);
 cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st);
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st);
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st);

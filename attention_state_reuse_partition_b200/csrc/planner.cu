@@ -1,0 +1,131 @@
+// Reductions of the anchor-guided planner (DiTango, arXiv 2607.15650; review
+// page, Referee Report major comments 1-3 and the Axiom & Free-Parameter
+// Ledger: Eq. 8 partition importance, Eq. 9 scale ratio, Eq. 10 local drift).
+//
+// Both kernels reduce in fp64 and in a fixed order: one CTA per
+// (partition i[, partition j], head bh) writes its partial sums to the scratch
+// buffer, and a second kernel adds the partials over bh in index order, so the
+// result does not depend on scheduling.
+//
+//   drift: for every partition i, sum over its rows (all b, h) of
+//          |now - anchor|^2 and |anchor|^2 (d columns each)
+//   stats: for every selected pair (i, j), sum over the rows of i of
+//          exp(LSE_ij - LSE_i) and |OUT_ij|^2
+#include "as_device.cuh"
+
+namespace asp {
+namespace {
+
+constexpr int THREADS = 256;
+
+__device__ __forceinline__ double block_sum(double x, double* sh) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) sh[warp] = x;
+  __syncthreads();
+  double tot = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < THREADS / 32; ++w) tot += sh[w];
+  return tot;  // valid in thread 0
+}
+
+// partials[(i * BH + bh) * 2 + {0, 1}]
+__global__ void __launch_bounds__(THREADS) drift_partials_kernel(const float* __restrict__ now,
+                                                                 const float* __restrict__ anchor, int BH, int S,
+                                                                 int d, int n, double* __restrict__ partials) {
+  __shared__ double sh[THREADS / 32];
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const long long base = (static_cast<long long>(bh) * S + static_cast<long long>(i) * n) * d;
+  const long long count = static_cast<long long>(n) * d;
+  double dd = 0.0, aa = 0.0;
+  for (long long e = threadIdx.x; e < count; e += THREADS) {
+    const double a = anchor[base + e];
+    const double x = now[base + e] - a;
+    dd += x * x;
+    aa += a * a;
+  }
+  const double sdd = block_sum(dd, sh);
+  const double saa = block_sum(aa, sh);
+  if (threadIdx.x == 0) {
+    partials[(static_cast<long long>(i) * BH + bh) * 2 + 0] = sdd;
+    partials[(static_cast<long long>(i) * BH + bh) * 2 + 1] = saa;
+  }
+}
+
+// partials[((i * P + j) * BH + bh) * 2 + {0, 1}] for selected pairs
+__global__ void __launch_bounds__(THREADS) stats_partials_kernel(const float* __restrict__ cache_out,
+                                                                 const float* __restrict__ cache_lse,
+                                                                 const float* __restrict__ lse_full,
+                                                                 long long plane_out, long long plane_lse, int P,
+                                                                 int BH, int S, int d, int n,
+                                                                 const __grid_constant__ PlanRows sel,
+                                                                 double* __restrict__ partials) {
+  __shared__ double sh[THREADS / 32];
+  const int pair = blockIdx.x, bh = blockIdx.y;
+  const int i = pair / P, j = pair % P;
+  if (!sel.v[pair]) {
+    if (threadIdx.x == 0) {
+      partials[(static_cast<long long>(pair) * BH + bh) * 2 + 0] = 0.0;
+      partials[(static_cast<long long>(pair) * BH + bh) * 2 + 1] = 0.0;
+    }
+    return;
+  }
+  const long long row0 = static_cast<long long>(bh) * S + static_cast<long long>(i) * n;
+  const float* lse_ij = cache_lse + j * plane_lse + row0;
+  const float* lse_i = lse_full + row0;
+  const float* out_ij = cache_out + j * plane_out + row0 * d;
+  double ws = 0.0, sq = 0.0;
+  for (int r = threadIdx.x; r < n; r += THREADS) ws += exp(static_cast<double>(lse_ij[r]) - lse_i[r]);
+  const long long count = static_cast<long long>(n) * d;
+  for (long long e = threadIdx.x; e < count; e += THREADS) {
+    const double o = out_ij[e];
+    sq += o * o;
+  }
+  const double sws = block_sum(ws, sh);
+  const double ssq = block_sum(sq, sh);
+  if (threadIdx.x == 0) {
+    partials[(static_cast<long long>(pair) * BH + bh) * 2 + 0] = sws;
+    partials[(static_cast<long long>(pair) * BH + bh) * 2 + 1] = ssq;
+  }
+}
+
+// out[k * 2 + c] = sum over bh of partials[(k * BH + bh) * 2 + c], in bh order
+__global__ void sum_over_heads_kernel(const double* __restrict__ partials, int K, int BH, double* __restrict__ out) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  double a = 0.0, b = 0.0;
+  for (int bh = 0; bh < BH; ++bh) {
+    a += partials[(static_cast<long long>(k) * BH + bh) * 2 + 0];
+    b += partials[(static_cast<long long>(k) * BH + bh) * 2 + 1];
+  }
+  out[k * 2 + 0] = a;
+  out[k * 2 + 1] = b;
+}
+
+}  // namespace
+
+cudaError_t launch_drift(const float* now, const float* anchor, int BH, int S, int d, int P, double* partials,
+                         double* sums, cudaStream_t st) {
+  const int n = S / P;
+  drift_partials_kernel<<<dim3(P, BH), THREADS, 0, st>>>(now, anchor, BH, S, d, n, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sum_over_heads_kernel<<<(P + 127) / 128, 128, 0, st>>>(partials, P, BH, sums);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_anchor_stats(const float* cache_out, const float* cache_lse, const float* lse_full,
+                                long long plane_out, long long plane_lse, int P, int BH, int S, int d,
+                                const PlanRows& sel, double* partials, double* sums, cudaStream_t st) {
+  const int n = S / P;
+  stats_partials_kernel<<<dim3(P * P, BH), THREADS, 0, st>>>(cache_out, cache_lse, lse_full, plane_out, plane_lse,
+                                                              P, BH, S, d, n, sel, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sum_over_heads_kernel<<<(P * P + 127) / 128, 128, 0, st>>>(partials, P * P, BH, sums);
+  return cudaGetLastError();
+}
+
+}  // namespace asp

@@ -409,6 +409,49 @@ def run_video_long(args, device):
     return {"workload": "video_long (4 steps)", "steps": per_step, "reuse_mse_vs_full_last_step": mse}
 
 
+def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5):
+    """Long video trajectory with the anchor-guided planner choosing each
+    step's plan: local states, drift, selection, the step, and the anchor
+    statistics after anchor steps."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec("video_long")
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    pl = api.AsPlanner(s.P, window, reuse_ratio, eps_local, s.B, s.H, s.S, s.d, device=device)
+    out = torch.empty((s.B, s.H, s.S, s.d), device=device)
+    lse = torch.empty((s.B, s.H, s.S), device=device)
+    local = torch.empty((s.B, s.H, s.S, s.d), device=device)
+    local_lse = torch.empty((s.B, s.H, s.S), device=device)
+    per_step = []
+    last = None
+    for t, q, k, v in W.video_trajectory(s, device=device):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        api.as_local_states(q, k, v, s.P, out=local, lse=local_lse)
+        plan, is_anchor, _ = api.as_planner_next(pl, local)          # synchronises
+        t1 = time.perf_counter()
+        api.as_step(cache, q, k, v, plan, t, out=out, lse=lse)
+        torch.cuda.synchronize()
+        t2 = time.perf_counter()
+        if is_anchor:
+            api.as_planner_commit_anchor(pl, cache, lse, plan)
+        t3 = time.perf_counter()
+        per_step.append({"step": t, "anchor": is_anchor, "planner_ms": round((t1 - t0) * 1e3, 3),
+                         "step_ms": round((t2 - t1) * 1e3, 3), "anchor_stats_ms": round((t3 - t2) * 1e3, 3),
+                         "reused_pairs": int((plan == W.PLAN_REUSE).sum()),
+                         "fresh_pairs": int((plan != W.PLAN_REUSE).sum()),
+                         "max_rel_drift": round(float(pl.rel_drift.max()), 5)})
+        last = (q, k, v)
+    q, k, v = last
+    full_o, _ = api.as_partition_attn(q, k, v, s.P, -1, list(range(s.P)))
+    torch.cuda.synchronize()
+    mse = torch.mean((out - full_o) ** 2).item()
+    del cache, pl, full_o, out, lse, local, local_lse, last, q, k, v
+    torch.cuda.empty_cache()
+    return {"workload": "video_long (4 steps) with the planner", "window": window, "reuse_ratio": reuse_ratio,
+            "eps_local": eps_local, "steps": per_step, "reuse_mse_vs_full_last_step": mse,
+            "timing": "wall clock around synchronising calls"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -418,7 +461,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
-    ap.add_argument("--only", choices=["compose", "reuse", "video_long"], default=None,
+    ap.add_argument("--only", choices=["compose", "reuse", "video_long", "planner"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
@@ -437,7 +480,8 @@ def main():
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if args.only is not None:
-        fn = {"compose": run_compose, "reuse": run_reuse, "video_long": run_video_long}[args.only]
+        fn = {"compose": run_compose, "reuse": run_reuse, "video_long": run_video_long,
+              "planner": run_planner}[args.only]
         print(json.dumps({"only": args.only, **fn(args, device)}))
         return
     if world > 1:
@@ -455,6 +499,7 @@ def main():
         secondary["compose"] = comp
         secondary["reuse"] = run_reuse(args, device)
         secondary["video_long"] = run_video_long(args, device)
+        secondary["planner"] = run_planner(args, device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.kernel_only:

@@ -150,6 +150,77 @@ as_status as_device_status(void* stream, uint32_t* h_bits);
  * usable.  Read the outcome with as_device_status. */
 as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * The anchor-guided planner (DiTango review: Referee Report major comments 1-3
+ * and the Axiom & Free-Parameter Ledger -- Eq. 7-10, 12, 13, Algorithm 1).
+ * Readings of the page:
+ *   w(i,j)     = mean over the rows of query partition i (all b, h) of
+ *                exp(LSE_ij - LSE_i), measured at an anchor (Eq. 8);
+ *   alpha(i,j) = ||OUT_ij||_F / ||OUT_ii||_F at the anchor (Eq. 9);
+ *   D(i,t)     = ||OUT_t(i,i) - OUT_ta(i,i)||_F, the local drift (Eq. 10);
+ *   ASE(i,j,t) = w(i,j) * alpha(i,j) * D(i,t) (Eq. 7, groups of one pair);
+ *   selection  : |i-j| <= window always fresh; of the other pairs, the
+ *                floor(R * count) with the smallest ASE are reused (ties by
+ *                (i, j)), the rest fresh and stored (Eq. 13, Algorithm 1);
+ *   anchor     : when there is none yet, or max_i D(i,t)/||OUT_ta(i,i)||_F >
+ *                eps_local; every pair fresh, every pair outside the window
+ *                stored.
+ * A step with the planner:
+ *   as_local_states(q,k,v,...) -> local_now            (device)
+ *   as_planner_next(pl, local_now, local_anchor, ...)  -> plan, is_anchor
+ *   as_step(cache, q,k,v, plan, ...)                   -> out, lse
+ *   if is_anchor: as_planner_commit_anchor(pl, cache, lse, local_anchor, plan, ...)
+ * ------------------------------------------------------------------------- */
+typedef struct as_planner {
+  uint32_t magic;
+  int P, window;
+  double reuse_ratio, eps_local;
+  int has_anchor;
+  double w[AS_MAX_P * AS_MAX_P];      /* w(i,j) of the last anchor (pairs outside the window) */
+  double alpha[AS_MAX_P * AS_MAX_P];  /* alpha(i,j) of the last anchor */
+  double drift[AS_MAX_P];             /* D(i,t) of the last as_planner_next (0 at anchors) */
+  double rel_drift[AS_MAX_P];         /* D(i,t) / ||OUT_ta(i,i)||_F */
+} as_planner;
+
+/* window >= 0, 0 <= reuse_ratio <= 1, eps_local >= 0, 1 <= P <= AS_MAX_P. */
+as_status as_planner_init(as_planner* pl, int P, int window, double reuse_ratio, double eps_local);
+
+/* Bytes of device scratch the planner reductions need (8-byte aligned buffer,
+ * caller-owned). */
+size_t as_planner_scratch_bytes(int B, int H, int P);
+
+/* The local (diagonal) states AS(i,i) of every query partition i in one
+ * launch: out [B,H,S,d], lse [B,H,S], partition i at rows [i n, (i+1) n).
+ * Same arguments and errors as as_partition_attn. */
+as_status as_local_states(const void* q, const void* k, const void* v, as_dtype dt, int B, int H, int S, int d,
+                          int P, float scale, float* out, float* lse, void* stream);
+
+/* For every partition i: h_drift[i] = ||now_i - anchor_i||_F and h_norm[i] =
+ * ||anchor_i||_F over its rows (all b, h, d), reduced in fp64 in a fixed
+ * order.  now, anchor [B,H,S,d] fp32 device.  Uses `scratch`; synchronises
+ * `stream` (the results are host values). */
+as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int S, int d, int P, void* scratch,
+                        size_t scratch_bytes, double* h_drift, double* h_norm, void* stream);
+
+/* Host-only selection from ASE values h_ase [P*P] (see the readings above). */
+as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan);
+
+/* Plan of the next step.  local_now: the step's local states (as_local_states);
+ * local_anchor [B,H,S,d]: the planner's copy of the anchor's local states,
+ * overwritten (stream-ordered copy) when this step becomes an anchor.  Writes
+ * h_plan [P*P], *h_is_anchor, and h_ase [P*P] (may be NULL; zeros at
+ * anchors).  Synchronises `stream`. */
+as_status as_planner_next(as_planner* pl, const float* local_now, float* local_anchor, int B, int H, int S, int d,
+                          void* scratch, size_t scratch_bytes, uint8_t* h_plan, int* h_is_anchor, double* h_ase,
+                          void* stream);
+
+/* After an anchor step (the as_step that used the anchor plan h_plan):
+ * measure w and alpha for every pair the plan stored, from the cache, the
+ * step's composed LSE lse_full [B,H,S] and local_anchor.  Synchronises. */
+as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const float* lse_full,
+                                   const float* local_anchor, const uint8_t* h_plan, void* scratch,
+                                   size_t scratch_bytes, void* stream);
+
 /* Test hook for the two exp2 evaluations the attention kernel mixes:
  * y[i] = 2^x[i] for n device floats, mode 0 = the FMA-pipe polynomial
  * (range reduction to [-1/2, 1/2], degree-4 minimax fit, relative error

@@ -140,3 +140,32 @@ def test_step_cache_miss_is_reported_before_any_launch(api):
     assert st == _lib.AS_ERR_CACHE_MISS
     assert "(0, 3)" in _lib.LIB.as_last_error().decode()
     assert (cache.t_c == -1).all()
+
+
+def test_plan_select_matches_fixture_and_oracle(api):
+    """The C selection against the hand-computed fixture and, bit-exactly, the
+    oracle's selection on random ASE values with ties."""
+    from oracle import as_oracle as O
+    from tests._golden import load_select_fixture
+    P, window, a, cases = load_select_fixture()
+    for ratio, plan in cases:
+        assert np.array_equal(api.as_plan_select(a, window, ratio), plan), ratio
+    r = np.random.default_rng(7)
+    for trial in range(40):
+        P = int(r.integers(1, 20))
+        window = int(r.integers(0, 4))
+        ase = np.round(r.random((P, P)) * 4) / 4  # many ties
+        ratio = float(r.choice([0.0, 0.1, 0.33, 0.5, 0.9, 1.0, r.random()]))
+        assert np.array_equal(api.as_plan_select(ase, window, ratio), O.select_plan(ase, window, ratio)), \
+            (P, window, ratio)
+
+
+def test_planner_init_validation(api):
+    from attention_state_reuse_partition_b200 import _lib
+    for args in [(0, 1, 0.5, 0.1), (65, 1, 0.5, 0.1), (4, -1, 0.5, 0.1), (4, 1, 1.5, 0.1), (4, 1, 0.5, -1.0)]:
+        with pytest.raises(api.AsError) as ei:
+            api.AsPlanner(*args)
+        assert ei.value.status == _lib.AS_ERR_INVALID_ARG
+    pl = api.AsPlanner(8, 2, 0.6, 0.05)
+    assert not pl.has_anchor and pl.P == 8
+    assert api.as_planner_scratch_bytes(1, 40, 32) == (32 * 32 * 40 * 2 + 32 * 32 * 2) * 8

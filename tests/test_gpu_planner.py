@@ -1,0 +1,152 @@
+"""The planner on the GPU against the float64 oracle.
+
+* local states: element-wise, with the bf16/fp32 tolerances of the parity
+  tests;
+* the drift and anchor-statistics reductions: on the same random fp32 inputs,
+  against float64 NumPy sums (relative 1e-9);
+* a planner trajectory: anchor decisions and plans against the oracle
+  planner.  Floating point decides these integers, so a pair whose oracle ASE
+  lies within a relative band of the selection threshold, or a step whose
+  relative drift lies within the band around eps_local, may legitimately go
+  either way; everything else must match exactly, and the states of query
+  partitions whose plan rows agree must match the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from attention_state_reuse_partition_b200 import workloads as W
+from oracle import as_oracle as O
+from tests.test_gpu_parity import check_bf16, check_f32, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    from attention_state_reuse_partition_b200 import build
+    build.build()
+    from attention_state_reuse_partition_b200 import api as a
+    return a
+
+
+def _oracle_local(qn, kn, vn, P, scale):
+    S = qn.shape[-2]
+    n = S // P
+    outs, lses = [], []
+    for i in range(P):
+        o, l = O.attention_state(qn[..., i * n:(i + 1) * n, :], kn[..., i * n:(i + 1) * n, :],
+                                 vn[..., i * n:(i + 1) * n, :], scale)
+        outs.append(o)
+        lses.append(l)
+    return np.concatenate(outs, axis=-2), np.concatenate(lses, axis=-1)
+
+
+@pytest.mark.parametrize("dtype,S,P", [("bf16", 16 * 8 * 16, 16), ("bf16", 5 * 192, 5), ("f32", 256, 4)])
+def test_local_states(api, dtype, S, P):
+    if dtype == "bf16":
+        s = W.spec("flux_image", H=2, S=S, P=P)
+        q, k, v = W.flux_qkv(s)
+        check = check_bf16
+    else:
+        s = W.spec("tiny_f32", P=P)
+        q, k, v = W.iid_qkv(s)
+        check = check_f32
+    out, lse = api.as_local_states(q.cuda(), k.cuda(), v.cuda(), P)
+    ref_o, ref_l = _oracle_local(f64(q), f64(k), f64(v), P, s.scale)
+    check(out, lse, ref_o, ref_l, f"local states {dtype} S={S} P={P}")
+
+
+def test_drift_reduction(api):
+    g = torch.Generator(device="cuda").manual_seed(11)
+    B, H, S, d, P = 1, 5, 640, 128, 5
+    now = torch.randn((B, H, S, d), generator=g, device="cuda")
+    anc = torch.randn((B, H, S, d), generator=g, device="cuda")
+    scratch = torch.empty(api.as_planner_scratch_bytes(B, H, P) // 8 + 1, dtype=torch.float64, device="cuda")
+    drift, norm = api.as_plan_drift(now, anc, P, scratch)
+    nn, aa = f64(now), f64(anc)
+    n = S // P
+    for i in range(P):
+        rd, rn = O.local_drift(nn[..., i * n:(i + 1) * n, :], aa[..., i * n:(i + 1) * n, :])
+        assert abs(drift[i] - rd) <= 1e-9 * rd and abs(norm[i] - rn) <= 1e-9 * rn
+
+
+def test_anchor_statistics(api):
+    """commit_anchor on a cache filled with known random states: w and alpha
+    of the stored pairs against float64 NumPy."""
+    B, H, S, d, P, window = 1, 3, 8 * 64, 64, 8, 1
+    n = S // P
+    cache = api.AsCache(B, H, S, d, P)
+    outs, lses = cache.planes()
+    g = torch.Generator(device="cuda").manual_seed(12)
+    outs.copy_(torch.randn(outs.shape, generator=g, device="cuda"))
+    lses.copy_(torch.randn(lses.shape, generator=g, device="cuda") + 2.0)
+    lse_full = torch.randn((B, H, S), generator=g, device="cuda") + 4.0
+    pl = api.AsPlanner(P, window, 0.5, 0.1, B, H, S, d)
+    pl.local_anchor.copy_(torch.randn((B, H, S, d), generator=g, device="cuda"))
+    plan = O.anchor_plan(P, window)
+    api.as_planner_commit_anchor(pl, cache, lse_full, plan)
+    assert pl.has_anchor
+    on, ln, lf, la = f64(outs), f64(lses), f64(lse_full), f64(pl.local_anchor)
+    for i in range(P):
+        local_norm = O.frob(la[..., i * n:(i + 1) * n, :])
+        for j in range(P):
+            if abs(i - j) <= window:
+                continue
+            w_ref = float(np.mean(np.exp(ln[j][..., i * n:(i + 1) * n] - lf[..., i * n:(i + 1) * n])))
+            a_ref = O.frob(on[j][..., i * n:(i + 1) * n, :]) / local_norm
+            assert abs(pl.w[i, j] - w_ref) <= 1e-9 * w_ref, (i, j)
+            assert abs(pl.alpha[i, j] - a_ref) <= 1e-9 * a_ref, (i, j)
+
+
+def test_planner_trajectory_against_oracle(api):
+    s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16, steps=6)
+    P, n, window, ratio, eps_local = s.P, s.n, 2, 0.6, 0.25
+    BAND = 1e-2
+    steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P)
+    pl = api.AsPlanner(P, window, ratio, eps_local, s.B, s.H, s.S, s.d)
+    ocache = O.StateCache(P)
+    opl = O.Planner(P, window, ratio, eps_local)
+    anchors = 0
+    for t, (q, k, v) in enumerate(steps):
+        qn, kn, vn = f64(q), f64(k), f64(v)
+        local, _ = api.as_local_states(q, k, v, P)
+        plan, is_anchor, ase = api.as_planner_next(pl, local)
+        olocal, _ = _oracle_local(qn, kn, vn, P, s.scale)
+        oplan, o_anchor, odrift, oase = O.planner_next(opl, olocal, n)
+        if t == 0:
+            assert is_anchor and o_anchor
+        else:
+            rel = np.array([odrift[i] / O.frob(opl.local_anchor[..., i * n:(i + 1) * n, :]) if not o_anchor else 0
+                            for i in range(P)])
+            if not o_anchor and abs(rel.max() - eps_local) > BAND * eps_local:
+                assert is_anchor == o_anchor, f"anchor decision at step {t}"
+        if is_anchor != o_anchor:
+            break  # an ambiguous anchor decision: the two trajectories part here
+        if not is_anchor:
+            remote = np.abs(np.arange(P)[:, None] - np.arange(P)[None, :]) > window
+            vals = np.sort(oase[remote])
+            k_reuse = int(np.floor(ratio * vals.size + 1e-9))
+            thr = vals[k_reuse - 1] if k_reuse > 0 else -np.inf
+            ambiguous = remote & (np.abs(oase - thr) <= BAND * max(abs(thr), 1e-30))
+            assert np.array_equal(plan[~ambiguous], oplan[~ambiguous]), f"plan at step {t}"
+            assert int((plan == O.PLAN_REUSE).sum()) == k_reuse
+        out, lse, hit, age = api.as_step(cache, q, k, v, plan, t)
+        torch.cuda.synchronize()
+        same_rows = [i for i in range(P) if np.array_equal(plan[i], oplan[i])]
+        ref_o, ref_l, _, _ = O.step(ocache, qn, kn, vn, oplan, t, s.scale)
+        for i in same_rows:
+            sl = slice(i * n, (i + 1) * n)
+            check_bf16(out[..., sl, :], lse[..., sl], ref_o[..., sl, :], ref_l[..., sl], f"step {t} partition {i}")
+        if is_anchor:
+            anchors += 1
+            api.as_planner_commit_anchor(pl, cache, lse, plan)
+            O.planner_commit_anchor(opl, ocache, ref_l, lambda i: np.arange(i * n, (i + 1) * n), n)
+            remote = np.abs(np.arange(P)[:, None] - np.arange(P)[None, :]) > window
+            assert np.allclose(pl.w[remote], opl.w[remote], rtol=5e-3, atol=0)
+            assert np.allclose(pl.alpha[remote], opl.alpha[remote], rtol=2e-2, atol=0)
+        if len(same_rows) < P:
+            break  # plans differ on an ambiguous pair: the caches part here
+    assert anchors >= 1
