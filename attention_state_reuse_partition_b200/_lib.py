@@ -23,7 +23,7 @@ STATUS_NAMES = {
 EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as_cache_bytes",
            "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe",
            "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
-           "as_plan_select", "as_planner_next", "as_planner_commit_anchor")
+           "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
     lib.as_local_states.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, ctypes.c_float, vp, vp, vp]
     lib.as_plan_drift.restype = c_int
     lib.as_plan_drift.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, vp, sz, vp, vp, vp]
+    lib.as_plan_drift_static.restype = c_int
+    lib.as_plan_drift_static.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, vp]
     lib.as_plan_select.restype = c_int
     lib.as_plan_select.argtypes = [vp, c_int, c_int, dbl, vp]
     lib.as_planner_next.restype = c_int

@@ -18,7 +18,7 @@ __all__ = ["as_partition_attn", "as_compose", "as_cache_bytes", "as_cache_init",
            "as_device_status", "as_debug_timeout_probe", "as_version", "AsCache", "AsError",
            "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE", "AsPlanner", "as_planner_init",
            "as_planner_scratch_bytes", "as_local_states", "as_plan_drift", "as_plan_select", "as_planner_next",
-           "as_planner_commit_anchor"]
+           "as_planner_commit_anchor", "as_plan_drift_static"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -239,6 +239,18 @@ def as_plan_drift(now, anchor, P: int, scratch, stream=None):
     check(LIB.as_plan_drift(_dev(now, "now"), _dev(anchor, "anchor"), B, H, S, d, P, _dev(scratch, "scratch"),
                             scratch.numel() * scratch.element_size(), drift.ctypes.data, norm.ctypes.data,
                             _stream_ptr(stream)))
+    return drift, norm
+
+
+def as_plan_drift_static(now, anchor, P: int, stream=None):
+    """as_plan_drift with the library's fixed scratch: for callers that cannot
+    allocate device memory (see include/as_partition.h).  The library
+    allocates nothing; the limit is P * (B*H*2 + 2) <= 131072."""
+    B, H, S, d = now.shape
+    drift = np.zeros(P, dtype=np.float64)
+    norm = np.zeros(P, dtype=np.float64)
+    check(LIB.as_plan_drift_static(_dev(now, "now"), _dev(anchor, "anchor"), B, H, S, d, P, drift.ctypes.data,
+                                   norm.ctypes.data, _stream_ptr(stream)))
     return drift, norm
 
 

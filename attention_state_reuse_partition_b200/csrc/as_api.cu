@@ -462,6 +462,41 @@ as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int
   return ok();
 }
 
+as_status as_plan_drift_static(const float* now, const float* anchor, int B, int H, int S, int d, int P,
+                               double* h_drift, double* h_norm, void* stream) {
+  as_status s = check_shape(B, H, S, d, P);
+  if (s != AS_OK) return s;
+  if (!now || !anchor || !h_drift || !h_norm) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_device()) != AS_OK) return s;
+  double* scratch = nullptr;
+  size_t capacity = 0;
+  cudaError_t e = asp::static_drift_scratch(&scratch, &capacity);
+  if (e != cudaSuccess) return cuda_fail(e, "fixed drift scratch address");
+  // partials [P][B*H][2] then sums [P][2]; every slot read is written first
+  // by the same call, so nothing needs clearing
+  const size_t need = static_cast<size_t>(P) * B * H * 2 + static_cast<size_t>(P) * 2;
+  if (need > capacity)
+    return fail(AS_ERR_INVALID_ARG,
+                "as_plan_drift_static: P*(B*H*2 + 2) = %zu doubles exceeds the fixed scratch of %zu doubles; "
+                "use as_plan_drift with a caller scratch buffer",
+                need, capacity);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  double* partials = scratch;
+  double* sums = scratch + static_cast<size_t>(P) * B * H * 2;
+  e = asp::launch_drift(now, anchor, B * H, S, d, P, partials, sums, st);
+  if (e != cudaSuccess) return cuda_fail(e, "drift launch");
+  std::vector<double> h(static_cast<size_t>(P) * 2);
+  e = cudaMemcpyAsync(h.data(), sums, h.size() * sizeof(double), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "drift copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "drift sync");
+  for (int i = 0; i < P; ++i) {
+    h_drift[i] = std::sqrt(h[i * 2 + 0]);
+    h_norm[i] = std::sqrt(h[i * 2 + 1]);
+  }
+  return ok();
+}
+
 as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan) {
   if (!h_ase || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
   if (P < 1 || P > AS_MAX_P || window < 0 || !(reuse_ratio >= 0.0 && reuse_ratio <= 1.0))

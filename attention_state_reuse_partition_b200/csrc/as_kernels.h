@@ -75,6 +75,8 @@ cudaError_t launch_attn_tc_bf16(const AttnLaunch& L, cudaStream_t st);
 // planner reductions: partials scratch [K][BH][2] doubles, sums [K][2] doubles
 cudaError_t launch_drift(const float* now, const float* anchor, int BH, int S, int d, int P, double* partials,
                          double* sums, cudaStream_t st);
+// address (on the current device) and size of the fixed drift scratch
+cudaError_t static_drift_scratch(double** ptr, size_t* capacity_doubles);
 cudaError_t launch_anchor_stats(const float* cache_out, const float* cache_lse, const float* lse_full,
                                 long long plane_out, long long plane_lse, int P, int BH, int S, int d,
                                 const PlanRows& sel, double* partials, double* sums, cudaStream_t st);

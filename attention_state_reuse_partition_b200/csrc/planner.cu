@@ -11,9 +11,18 @@
 //          |now - anchor|^2 and |anchor|^2 (d columns each)
 //   stats: for every selected pair (i, j), sum over the rows of i of
 //          exp(LSE_ij - LSE_i) and |OUT_ij|^2
+#include <mutex>
+
 #include "as_device.cuh"
 
 namespace asp {
+
+// Fixed scratch for the allocation-free drift entry point
+// (as_plan_drift_static): partials [P][B*H][2] doubles, then sums [P][2].
+// 1 MiB, held by every device that loads the library until the process exits.
+constexpr size_t STATIC_DRIFT_DOUBLES = size_t(1) << 17;
+static __device__ __align__(256) double g_static_drift_scratch[STATIC_DRIFT_DOUBLES];
+
 namespace {
 
 constexpr int THREADS = 256;
@@ -114,6 +123,30 @@ cudaError_t launch_drift(const float* now, const float* anchor, int BH, int S, i
   if (e != cudaSuccess) return e;
   sum_over_heads_kernel<<<(P + 127) / 128, 128, 0, st>>>(partials, P, BH, sums);
   return cudaGetLastError();
+}
+
+// Device address of the fixed drift scratch on the current device.  In host
+// code the array's name only stands in for the symbol, so the address comes
+// from cudaGetSymbolAddress, once per device (the first call on a device does
+// it, with that device current), and is cached.
+cudaError_t static_drift_scratch(double** ptr, size_t* capacity_doubles) {
+  constexpr int MAX_DEVICES = 64;
+  static double* addr[MAX_DEVICES] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_drift_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<double*>(p);
+  }
+  *ptr = addr[dev];
+  *capacity_doubles = STATIC_DRIFT_DOUBLES;
+  return cudaSuccess;
 }
 
 cudaError_t launch_anchor_stats(const float* cache_out, const float* cache_lse, const float* lse_full,

@@ -202,6 +202,27 @@ as_status as_local_states(const void* q, const void* k, const void* v, as_dtype 
 as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int S, int d, int P, void* scratch,
                         size_t scratch_bytes, double* h_drift, double* h_norm, void* stream);
 
+/* as_plan_drift without a scratch argument, for callers that cannot allocate
+ * device memory: a host that owns every device allocation itself and hands
+ * this library only fixed, pre-sized buffers, or a loop that must not
+ * allocate once running (cudaMalloc may synchronise the device and can fail
+ * under memory pressure), and so cannot provide the scratch buffer that
+ * as_plan_drift needs.  The paper has no counterpart: this is an interface
+ * variant, not a step of the method.
+ *   Same arguments, results and synchronisation as as_plan_drift.  The
+ *   scratch is a fixed 1 MiB array inside the library (held on every device
+ *   that loads it until the process exits); the call allocates nothing.
+ *   Limit: P * (B*H*2 + 2) <= 131072 doubles, else AS_ERR_INVALID_ARG with the
+ *   sizes in as_last_error().
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call uses the same array and leaves its contents behind; each call
+ *   writes every slot it reads, so nothing has to be cleared.  Calls that
+ *   overlap on the GPU (different streams, or different host threads on one
+ *   device) race on the array: serialise them. */
+as_status as_plan_drift_static(const float* now, const float* anchor, int B, int H, int S, int d, int P,
+                               double* h_drift, double* h_norm, void* stream);
+
 /* Host-only selection from ASE values h_ase [P*P] (see the readings above). */
 as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan);
 
