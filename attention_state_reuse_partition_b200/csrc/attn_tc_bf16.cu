@@ -23,9 +23,13 @@
 // MMAs ahead of the tensor core), so the tensor core works on one tile while
 // the other tile's softmax runs.  A commit after QK_t completes only when
 // every earlier MMA has, so when the softmax of tile t sees S_t its previous
-// PV has finished: O_t may be rescaled and P_t written without a further wait.  O is rescaled only when a row maximum grows by more than 2^8;
-// OUT and the row sum share the same reference maximum, so the result is
-// unchanged.
+// PV has finished: O_t may be rescaled and P_t written without a further
+// wait.  O is rescaled only when a row maximum grows by more than 2^8; OUT and
+// the row sum share the same reference maximum, so the result is unchanged.
+// At a group end each softmax warp moves its 32 rows of O through a small
+// shared-memory block, 16 columns at a time, so that the global stores write
+// whole row segments; O_t is released to the next group as soon as it has
+// been read.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -78,11 +82,20 @@ struct Ctrl {
   KvSchedule sched;
 };
 
+// Output staging: each softmax warp transposes its 32 rows through a
+// 32 x 16-float block (row stride STAGE_LD floats: the float4 writes of 8
+// consecutive rows cover all 32 banks), so that each global store
+// instruction writes whole 64-byte row segments instead of 32 scattered
+// 16-byte pieces.
+constexpr int STAGE_LD = 20;
+constexpr int STAGE_FLOATS = 32 * STAGE_LD;  // per softmax warp
+constexpr int CTRL_BYTES = (static_cast<int>(sizeof(Ctrl)) + 15) & ~15;
+
 template <int D>
 constexpr int smem_bytes() {
   // at least 116 KB so that only one CTA (and one 512-column TMEM allocation)
   // fits on an SM
-  constexpr int need = Layout<D>::CTRL_OFF + static_cast<int>(sizeof(Ctrl)) + 1024;
+  constexpr int need = Layout<D>::CTRL_OFF + CTRL_BYTES + 4 * NQ * STAGE_FLOATS * 4 + 1024;
   return need > 116 * 1024 ? need : 116 * 1024;
 }
 
@@ -396,6 +409,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         f2_unpack(p2, p0, p1);
         pk[i] = pack_bf16x2(p0, p1);
       }
+      // the previous PV of this tile has completed (see the header), so P may
+      // be written over S and O rescaled now; P goes first, which frees its
+      // registers for the rescale
+      tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int ch = 0; ch < D / 16; ++ch) {
+          uint32_t r[16];
+          tmem_ld16(t_lane + o_col + ch * 16, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(t_lane + o_col + ch * 16, r);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&c.p_full[t]);
       float rs;
       {
         const uint64_t a = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
@@ -403,60 +435,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         f2_unpack(a, lo, hi);
         rs = lo + hi;
       }
-      // the previous PV of this tile has completed (see the header), so O may
-      // be rescaled and P written over S now
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + o_col + ch * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(t_lane + o_col + ch * 32, r);
-        }
-      }
-      tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&c.p_full[t]);
       l = first ? rs : fmaf(l, alpha, rs);
       m = m_use;
       if (last) {
         if (!warp_wait(&c.o_ready[t], group & 1, abort_flag, budget)) break;
         tc_fence_after();
+        // the warp's 32 rows are consecutive in the destination: s_row0 + rr
+        const int s_row0 = s_row - lane;
         const int dest = c.sched.group_dest[group];
-        float* orow;
+        float* orow0;  // row s_row0
         float* lrow;
         if (dest < 0) {
-          const long long r_idx = static_cast<long long>(bh) * L.out_rows + (s_row - L.out_row0);
-          orow = L.out + r_idx * D;
-          lrow = L.lse + r_idx;
+          const long long r_idx = static_cast<long long>(bh) * L.out_rows + (s_row0 - L.out_row0);
+          orow0 = L.out + r_idx * D;
+          lrow = L.lse + r_idx + lane;
         } else {
-          const long long r_idx = static_cast<long long>(bh) * L.dst_rows + (s_row - L.dst_row0);
-          orow = L.dst_out + dest * L.dst_plane_out + r_idx * D;
-          lrow = L.dst_lse + dest * L.dst_plane_lse + r_idx;
+          const long long r_idx = static_cast<long long>(bh) * L.dst_rows + (s_row0 - L.dst_row0);
+          orow0 = L.dst_out + dest * L.dst_plane_out + r_idx * D;
+          lrow = L.dst_lse + dest * L.dst_plane_lse + r_idx + lane;
         }
-        const bool write = s_row < q_hi;
         const float inv_l = 1.0f / l;
+        float* stage = reinterpret_cast<float*>(smem + Lay::CTRL_OFF + CTRL_BYTES) + (warp - 4) * STAGE_FLOATS;
+        // read-back role of this lane: rows rr = 8 i + lane / 4, columns 4 (lane % 4) .. + 3
+        const int rb_row = lane >> 2, rb_col = (lane & 3) * 4;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + o_col + ch * 32, r);
+        for (int ch = 0; ch < D / 16; ++ch) {
+          uint32_t r[16];
+          tmem_ld16(t_lane + o_col + ch * 16, r);
           tmem_wait_ld();
-          if (write) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              float4 o4 = make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
-                                      __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
-              *reinterpret_cast<float4*>(orow + ch * 32 + e) = o4;
-            }
+          if (ch == D / 16 - 1) {
+            // O has been read: the next group may overwrite it
+            tc_fence_before();
+            mbar_arrive(&c.o_free[t]);
           }
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(stage + lane * STAGE_LD + e) =
+                make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                            __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 8 * i + rb_row;
+            const float4 v4 = *reinterpret_cast<const float4*>(stage + rr * STAGE_LD + rb_col);
+            if (s_row0 + rr < q_hi)
+              *reinterpret_cast<float4*>(orow0 + static_cast<long long>(rr) * D + ch * 16 + rb_col) = v4;
+          }
+          __syncwarp();
         }
-        if (write) *lrow = (m + log2f(l)) * 0.6931471805599453f;
-        tc_fence_before();
-        mbar_arrive(&c.o_free[t]);
+        if (s_row < q_hi) *lrow = (m + log2f(l)) * 0.6931471805599453f;
       }
     }
     tc_fence_before();
