@@ -27,6 +27,16 @@ contiguous, equal and in token order; the empty state is (OUT=0, LSE=-inf); a
 plan entry is 0=reuse, 1=fresh, 2=fresh and refresh the cached entry; hit is 1
 exactly for reused pairs and age = t - t_c for them (0 otherwise).
 
+Memory-aware merging (review page, "If this is right", second bullet: composed
+states "can be merged into coarser groups under memory pressure"; ledger:
+group size g = 4/8/16): KV partition j belongs to group j // g, and the cache
+holds one composed state per (query partition i, group G) together with the
+set of members it was composed from.  A group is refreshed or reused as a
+whole; a reuse must name exactly the stored members.  Entries may keep OUT in
+bf16 (round to nearest even from fp32); the LSE stays fp32.  A step composes
+what the cache holds, so at a store step the stored groups enter the final
+state with the cache's precision.
+
 Every pin of this module lives in ``tests/test_oracle.py``.
 """
 from __future__ import annotations
@@ -39,11 +49,23 @@ PLAN_FRESH_STORE = 2
 
 
 class CacheMiss(Exception):
-    """A plan reuses a pair whose cache entry has never been written."""
+    """A plan reuses a pair whose cache entry has never been written, or (with
+    groups) reuses a member set other than the one stored."""
 
 
 class PlanError(Exception):
-    """A plan matrix holds a value other than 0, 1 or 2, or has a wrong shape."""
+    """A plan matrix holds a value other than 0, 1 or 2, has a wrong shape, or
+    (with groups) both reuses and stores members of one group."""
+
+
+def round_bf16(x):
+    """Round to bfloat16 and back: float64 -> float32 (nearest even), then the
+    low 16 bits of the float32 rounded off to nearest even.  Finite inputs."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> np.uint64(16)) & np.uint64(1)
+    bits = (bits + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
+    return bits.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
 # ---------------------------------------------------------------------------
@@ -148,52 +170,90 @@ def full_attention(q, k, v, scale):
 # plan resolution and the state cache
 # ---------------------------------------------------------------------------
 
-def resolve_plan(plan, t_c, t):
+def n_groups(P, g):
+    """Number of KV groups of size g over P partitions (the last may be short)."""
+    return (P + g - 1) // g
+
+
+def resolve_plan(plan, t_c, t, g=1, member=None):
     """Check a plan against the cache timestamps and derive hit and age.
 
     plan [P,P] uint8 (row i = query partition, column j = KV partition), t_c
-    [P,P] int (step of the entry's last write, -1 = never written), t the
-    current step.  hit[i,j] = 1 for reused pairs, else 0; age[i,j] = t - t_c
-    for reused pairs, else 0.  A reuse of a never-written entry raises
-    CacheMiss; any other value than 0/1/2 raises PlanError.
+    [P, n_groups(P, g)] int (step of the entry's last write, -1 = never
+    written), t the current step.  hit[i,j] = 1 for reused pairs, else 0;
+    age[i,j] = t - t_c[i, j // g] for reused pairs, else 0.  A reuse of a
+    never-written entry raises CacheMiss, and so does a reuse whose member set
+    differs from ``member[i][G]`` (the members stored, when given); a group
+    with both reused and stored members, or any value other than 0/1/2,
+    raises PlanError.  With g = 1 each pair is its own group.
     """
     plan = np.asarray(plan)
     t_c = np.asarray(t_c)
     P = plan.shape[0]
-    if plan.ndim != 2 or plan.shape != (P, P) or t_c.shape != (P, P):
-        raise PlanError("plan and t_c must both be [P, P]")
-    hit = np.zeros((P, P), dtype=np.uint8)
-    age = np.zeros((P, P), dtype=np.int32)
+    NG = n_groups(P, g)
+    if plan.ndim != 2 or plan.shape != (P, P) or t_c.shape != (P, NG):
+        raise PlanError("plan must be [P, P] and t_c [P, n_groups]")
     for i in range(P):
         for j in range(P):
-            c = int(plan[i, j])
-            if c not in (PLAN_REUSE, PLAN_FRESH, PLAN_FRESH_STORE):
-                raise PlanError(f"plan[{i},{j}] = {c}")
-            if c == PLAN_REUSE:
-                if t_c[i, j] < 0:
-                    raise CacheMiss(f"pair ({i},{j}) reused before any store")
+            if int(plan[i, j]) not in (PLAN_REUSE, PLAN_FRESH, PLAN_FRESH_STORE):
+                raise PlanError(f"plan[{i},{j}] = {int(plan[i, j])}")
+    hit = np.zeros((P, P), dtype=np.uint8)
+    age = np.zeros((P, P), dtype=np.int32)
+
+    def members(i, G, code):
+        return frozenset(j for j in range(G * g, min((G + 1) * g, P)) if int(plan[i, j]) == code)
+
+    for i in range(P):
+        for G in range(NG):
+            if members(i, G, PLAN_REUSE) and members(i, G, PLAN_FRESH_STORE):
+                raise PlanError(f"group ({i},{G}) both reuses and stores members")
+    for i in range(P):
+        for G in range(NG):
+            reused = members(i, G, PLAN_REUSE)
+            if not reused:
+                continue
+            if t_c[i, G] < 0:
+                raise CacheMiss(f"group ({i},{G}) reused before any store")
+            if member is not None and reused != member[i][G]:
+                raise CacheMiss(f"group ({i},{G}) reuses members {sorted(reused)}, "
+                                f"stored {sorted(member[i][G])}")
+            for j in reused:
                 hit[i, j] = 1
-                age[i, j] = t - int(t_c[i, j])
+                age[i, j] = t - int(t_c[i, G])
     return hit, age
 
 
 class StateCache:
-    """One cached state per (query partition i, KV partition j), for the query
-    rows the oracle evaluates, plus the step t_c of each entry's last write."""
+    """One cached state per (query partition i, KV group G) for the query rows
+    the oracle evaluates, the member set it was composed from, and the step
+    t_c of its last write.  g = 1 and cache_dt "f32" give one exact entry per
+    pair; cache_dt "bf16" keeps OUT rounded to bf16."""
 
-    def __init__(self, P):
-        self.P = P
-        self.t_c = np.full((P, P), -1, dtype=np.int64)
+    def __init__(self, P, g=1, cache_dt="f32"):
+        if g < 1 or g > P:
+            raise PlanError(f"group size {g} outside [1, {P}]")
+        if cache_dt not in ("f32", "bf16"):
+            raise PlanError(f"cache dtype {cache_dt}")
+        self.P, self.g, self.cache_dt = P, g, cache_dt
+        self.NG = n_groups(P, g)
+        self.t_c = np.full((P, self.NG), -1, dtype=np.int64)
+        self.member = [[frozenset() for _ in range(self.NG)] for _ in range(P)]
         self.entry = {}
 
 
 def step(cache, q, k, v, plan, t, scale, rows=None):
     """One denoising step's attention under a compute/reuse plan.
 
-    final(i) = compose({AS_t(i,j) : plan[i,j] fresh} U {C(i,j) : plan[i,j] = reuse}),
-    then C(i,j) <- AS_t(i,j) and t_c(i,j) <- t for plan[i,j] = fresh-and-store.
-    (DiTango review: Core claim and Referee Report Summary -- fresh states for
-    near partitions, cached composed states from earlier steps for far ones.)
+    final(i) = compose({AS_t(i,j) : plan[i,j] = fresh}
+                       U {C(i,G) : G stored at this step}
+                       U {C(i,G) : G reused}),
+    where a stored group's entry C(i,G) <- compose({AS_t(i,j) : plan[i,j] =
+    fresh-and-store, j in G}) (OUT rounded to the cache dtype), member(i,G)
+    <- those j, and t_c(i,G) <- t.  (DiTango review: Core claim and Referee
+    Report Summary -- fresh states for near partitions, cached composed
+    states from earlier steps for far ones; "If this is right" -- composed
+    states merged into coarser groups.)  With g = 1 and an fp32 cache this is
+    compose of every pair's fresh state or cached entry.
 
     q, k, v: [B,H,S,d].  ``rows``: sorted token indices of the query rows to
     evaluate (default all); the same rows must be used at every step of one
@@ -202,10 +262,10 @@ def step(cache, q, k, v, plan, t, scale, rows=None):
     """
     q = np.asarray(q, dtype=np.float64)
     S = k.shape[-2]
-    P = cache.P
+    P, g = cache.P, cache.g
     n = S // P
     rows = np.arange(S) if rows is None else np.asarray(rows)
-    hit, age = resolve_plan(plan, cache.t_c, t)
+    hit, age = resolve_plan(plan, cache.t_c, t, g, cache.member)
     B, H, _, d = q.shape
     out = np.zeros((B, H, len(rows), d))
     lse = np.zeros((B, H, len(rows)))
@@ -217,21 +277,37 @@ def step(cache, q, k, v, plan, t, scale, rows=None):
             continue
         qi = q[:, :, rows[sel], :]
         parts = []
-        for j, (a, b) in enumerate(bounds):
-            c = int(plan[i, j])
-            if c == PLAN_REUSE:
-                parts.append(cache.entry[(i, j)])
-            else:
+        for G in range(cache.NG):
+            js = range(G * g, min((G + 1) * g, P))
+            to_store = []
+            reused = False
+            for j in js:
+                c = int(plan[i, j])
+                if c == PLAN_REUSE:
+                    reused = True
+                    continue
+                a, b = bounds[j]
                 st = attention_state(qi, k[..., a:b, :], v[..., a:b, :], scale)
-                parts.append(st)
                 if c == PLAN_FRESH_STORE:
-                    updates.append(((i, j), st))
+                    to_store.append(st)
+                else:
+                    parts.append(st)
+            if reused:
+                parts.append(cache.entry[(i, G)])
+            if to_store:
+                o, l = compose(to_store)
+                if cache.cache_dt == "bf16":
+                    o = round_bf16(o)
+                parts.append((o, l))
+                members = frozenset(j for j in js if int(plan[i, j]) == PLAN_FRESH_STORE)
+                updates.append(((i, G), (o, l), members))
         o, l = compose(parts)
         out[:, :, sel, :] = o
         lse[:, :, sel] = l
-    for key, st in updates:
+    for key, st, members in updates:
         cache.entry[key] = st
         cache.t_c[key] = t
+        cache.member[key[0]][key[1]] = members
     return out, lse, hit, age
 
 

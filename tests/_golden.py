@@ -10,12 +10,16 @@ def _matrix(lines, P, dtype):
     return np.array([[int(x) for x in lines.pop(0).split()] for _ in range(P)], dtype=dtype)
 
 
-def load_plan_fixture(name="plan_4x4.txt"):
-    """Returns (P, [dict(step, plan, expect, hit, age)])."""
+def load_plan_fixture(name="plan_4x4.txt", with_group=False):
+    """Returns (P, [dict(step, plan, expect, hit, age)]), or (P, g, cases)
+    with ``with_group`` (a fixture without a "g" line has g = 1)."""
     with open(os.path.join(GOLDEN, name)) as f:
         lines = [ln.strip() for ln in f if ln.strip() and not ln.lstrip().startswith("#")]
     assert lines[0].startswith("P ")
     P = int(lines.pop(0).split()[1])
+    g = 1
+    if lines[0].startswith("g "):
+        g = int(lines.pop(0).split()[1])
     cases = []
     while lines:
         head = lines.pop(0)
@@ -30,6 +34,8 @@ def load_plan_fixture(name="plan_4x4.txt"):
             assert lines.pop(0) == "age"
             case["age"] = _matrix(lines, P, np.int32)
         cases.append(case)
+    if with_group:
+        return P, g, cases
     return P, cases
 
 

@@ -42,6 +42,16 @@ def _sdpa(q, k, v, scale):
     return out.numpy()
 
 
+def _expect_raises(exc, fn, *args, **kw):
+    """Like pytest.raises, but a miss is an AssertionError (an Exception), so
+    the planted-mistake harness sees it."""
+    try:
+        fn(*args, **kw)
+    except exc:
+        return
+    raise AssertionError(f"{exc.__name__} not raised")
+
+
 def _close(a, b, tol=TOL, what=""):
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
@@ -184,13 +194,11 @@ def pin_plan_golden(o):
     for c in cases:
         if c["expect"] == "cache_miss":
             before = cache.t_c.copy()
-            with pytest.raises(o.CacheMiss):
-                o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
+            _expect_raises(o.CacheMiss, o.step, cache, q, k, v, c["plan"], c["step"], 0.5)
             assert np.array_equal(cache.t_c, before), "cache changed on a miss"
             continue
         if c["expect"] == "invalid":
-            with pytest.raises(o.PlanError):
-                o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
+            _expect_raises(o.PlanError, o.step, cache, q, k, v, c["plan"], c["step"], 0.5)
             continue
         _, _, hit, age = o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
         assert np.array_equal(hit, c["hit"]), f"hit at step {c['step']}"
@@ -261,6 +269,104 @@ def pin_step_reuse_mixed(o):
         ref = _sdpa(q[..., row:row + 1, :], km, vm, 0.4)[..., 0, :]
         _close(out[:, :, idx, :], ref, TOL, f"mixed row {row}")
     assert cache.t_c[0, 4] == 1 and cache.t_c[0, 3] == 0
+
+
+# ---------------------------------------------------------------------------
+# grouped cache and bf16 entries (DiTango review: "If this is right" -- merged
+# composed states under memory pressure; ledger: group size g)
+# ---------------------------------------------------------------------------
+
+def pin_round_bf16(o):
+    """bf16 rounding against torch's float32 -> bfloat16 conversion (round to
+    nearest even), on random magnitudes and on exact halfway cases."""
+    r = _rng(30)
+    x = np.concatenate([r.normal(size=2000) * 10.0 ** r.integers(-6, 6, size=2000),
+                        [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 0.0, -0.0, 1.5, 2.0 ** -100]])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    got = o.round_bf16(x)
+    assert np.array_equal(got, ref), f"bf16 rounding differs at {np.nonzero(got != ref)[0][:5]}"
+    assert o.round_bf16(1.0 + 2.0 ** -8) == 1.0 and o.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+
+
+def pin_plan_grouped_golden(o):
+    P, g, cases = load_plan_fixture("plan_grouped_4x4.txt", with_group=True)
+    r = _rng(31)
+    S, d = 2 * P, 3
+    q, k, v = (r.normal(size=(1, 1, S, d)) for _ in range(3))
+    cache = o.StateCache(P, g)
+    for c in cases:
+        if c["expect"] in ("cache_miss", "invalid"):
+            before = (cache.t_c.copy(), [list(m) for m in cache.member])
+            _expect_raises(o.CacheMiss if c["expect"] == "cache_miss" else o.PlanError,
+                           o.step, cache, q, k, v, c["plan"], c["step"], 0.5)
+            assert np.array_equal(cache.t_c, before[0]) and cache.member == before[1], "cache changed on an error"
+            continue
+        _, _, hit, age = o.step(cache, q, k, v, c["plan"], c["step"], 0.5)
+        assert np.array_equal(hit, c["hit"]), f"grouped hit at step {c['step']}"
+        assert np.array_equal(age, c["age"]), f"grouped age at step {c['step']}"
+
+
+def pin_step_grouped_identical(o):
+    """Window plans with grouped entries (g = 2, 3, 4 over P = 6, the last
+    group short for g = 4): reusing entries of unchanged inputs gives full
+    attention (sdpa), and hit/age follow the pairs."""
+    r = _rng(32)
+    B, H, S, d, P = 1, 2, 48, 8, 6
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    anchor, reuse = _window_plans(P, 1)
+    for g in (2, 3, 4):
+        cache = o.StateCache(P, g)
+        out0, _, _, _ = o.step(cache, q, k, v, anchor, 0, 0.3)
+        _close(out0, _sdpa(q, k, v, 0.3), TOL, f"grouped anchor g={g}")
+        assert cache.t_c.shape == (P, (P + g - 1) // g)
+        out, _, hit, age = o.step(cache, q, k, v, reuse, 1, 0.3)
+        _close(out, _sdpa(q, k, v, 0.3), TOL, f"grouped reuse g={g}")
+        assert np.array_equal(hit, (reuse == 0).astype(np.uint8)) and np.array_equal(age, hit.astype(np.int32))
+
+
+def pin_step_grouped_mixed(o):
+    """K/V move between steps; a reused group must carry the step-0 K/V of
+    exactly its stored members, so each row equals sdpa over K/V stitched per
+    partition.  Row 0 refreshes its far group at step 1."""
+    r = _rng(33)
+    B, H, S, d, P, g = 1, 2, 48, 8, 6, 2
+    n = S // P
+    q = r.normal(size=(B, H, S, d))
+    k0, v0 = r.normal(size=(B, H, S, d)), r.normal(size=(B, H, S, d))
+    k1, v1 = k0 + r.normal(size=k0.shape), v0 + r.normal(size=v0.shape)
+    anchor, reuse = _window_plans(P, 1)
+    reuse[0, 4:6] = o_STORE
+    cache = o.StateCache(P, g)
+    rows = np.array([1, 9, 15, 22, 30, 37, 41, 47])  # every partition has rows
+    o.step(cache, q, k0, v0, anchor, 0, 0.4, rows=rows)
+    out, _, _, _ = o.step(cache, q, k1, v1, reuse, 1, 0.4, rows=rows)
+    for idx, row in enumerate(rows):
+        i = row // n
+        km, vm = k0.copy(), v0.copy()
+        for j in range(P):
+            if reuse[i, j] != o_REUSE:
+                km[..., j * n:(j + 1) * n, :] = k1[..., j * n:(j + 1) * n, :]
+                vm[..., j * n:(j + 1) * n, :] = v1[..., j * n:(j + 1) * n, :]
+        _close(out[:, :, idx, :], _sdpa(q[..., row:row + 1, :], km, vm, 0.4)[..., 0, :], TOL, f"grouped row {row}")
+    assert cache.t_c[0, 2] == 1 and cache.t_c[1, 2] == 0 and cache.member[0][2] == frozenset({4, 5})
+
+
+def pin_step_bf16_cache(o):
+    """bf16 entries: a reuse of unchanged inputs differs from full attention
+    by no more than the rounding of the reused OUT (relative 2^-8 of its
+    magnitude), and it does differ (the entries are rounded)."""
+    r = _rng(34)
+    B, H, S, d, P = 1, 2, 48, 8, 6
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    anchor, reuse = _window_plans(P, 1)
+    ref = _sdpa(q, k, v, 0.3)
+    for g in (1, 3):
+        cache = o.StateCache(P, g, "bf16")
+        o.step(cache, q, k, v, anchor, 0, 0.3)
+        out, _, _, _ = o.step(cache, q, k, v, reuse, 1, 0.3)
+        bound = 2.0 ** -8 * max(float(np.max(np.abs(e[0]))) for e in cache.entry.values())
+        err = float(np.max(np.abs(out - ref)))
+        assert 0.0 < err <= bound, f"bf16 cache g={g}: err {err}, bound {bound}"
 
 
 # ---------------------------------------------------------------------------
@@ -354,7 +460,9 @@ def pin_planner_trajectory(o):
 PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_forms,
         pin_compose_closed, pin_assoc_comm, pin_split_invariance, pin_single_partition,
         pin_plan_golden, pin_step_all_fresh, pin_step_reuse_identical, pin_step_reuse_mixed,
-        pin_planner_weights, pin_planner_ratios, pin_planner_drift, pin_planner_select, pin_planner_trajectory]
+        pin_planner_weights, pin_planner_ratios, pin_planner_drift, pin_planner_select, pin_planner_trajectory,
+        pin_round_bf16, pin_plan_grouped_golden, pin_step_grouped_identical, pin_step_grouped_mixed,
+        pin_step_bf16_cache]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -368,7 +476,7 @@ def test_oracle_passes_pin(pin):
 
 _orig = {name: getattr(as_oracle, name) for name in
          ("attention_state", "compose", "compose_pair", "resolve_plan", "step", "partition_bounds",
-          "anchor_weights", "scale_ratios", "local_drift", "select_plan", "ase")}
+          "anchor_weights", "scale_ratios", "local_drift", "select_plan", "ase", "round_bf16", "n_groups")}
 
 
 def _m_no_normalise(q, k, v, scale):
@@ -421,14 +529,44 @@ def _m_pair_max_only(a, b):
     return out, np.maximum(a[1], b[1])
 
 
-def _m_age_sign(plan, t_c, t):
-    hit, age = _orig["resolve_plan"](plan, t_c, t)
+def _m_age_sign(plan, t_c, t, g=1, member=None):
+    hit, age = _orig["resolve_plan"](plan, t_c, t, g, member)
     return hit, -age
 
 
-def _m_hit_fresh(plan, t_c, t):
-    hit, age = _orig["resolve_plan"](plan, t_c, t)
+def _m_hit_fresh(plan, t_c, t, g=1, member=None):
+    hit, age = _orig["resolve_plan"](plan, t_c, t, g, member)
     return (1 - hit).astype(np.uint8), age
+
+
+def _m_members_unchecked(plan, t_c, t, g=1, member=None):
+    return _orig["resolve_plan"](plan, t_c, t, g, None)
+
+
+def _m_group_stores_fresh_members(cache, q, k, v, plan, t, scale, rows=None):
+    plan2 = np.array(plan, dtype=np.uint8, copy=True)
+    P, g = cache.P, cache.g
+    for i in range(P):
+        for G in range((P + g - 1) // g):
+            js = range(G * g, min((G + 1) * g, P))
+            if any(plan2[i, j] == 2 for j in js):
+                for j in js:
+                    if plan2[i, j] == 1:
+                        plan2[i, j] = 2
+    return _orig["step"](cache, q, k, v, plan2, t, scale, rows)
+
+
+def _m_bf16_truncate(x):
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    return (f.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+
+
+def _m_bf16_not_rounded(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _m_groups_floor(P, g):
+    return P // g
 
 
 def _m_store_all_fresh(cache, q, k, v, plan, t, scale, rows=None):
@@ -489,6 +627,11 @@ MUTANTS = {
     "select_plan: reuses the largest ASE": ("select_plan", _m_select_largest),
     "select_plan: window off by one": ("select_plan", _m_select_window),
     "ase: drops the scale ratio": ("ase", _m_ase_no_alpha),
+    "resolve_plan: reused member set not checked": ("resolve_plan", _m_members_unchecked),
+    "step: a stored group takes its plain-fresh members too": ("step", _m_group_stores_fresh_members),
+    "round_bf16: truncates": ("round_bf16", _m_bf16_truncate),
+    "round_bf16: no rounding": ("round_bf16", _m_bf16_not_rounded),
+    "n_groups: drops the short last group": ("n_groups", _m_groups_floor),
 }
 
 
