@@ -23,7 +23,8 @@ STATUS_NAMES = {
 EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as_cache_bytes",
            "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe",
            "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
-           "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static")
+           "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static",
+           "as_cache_group_bytes", "as_cache_group_init")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -34,6 +35,8 @@ class AsCacheStruct(ctypes.Structure):
         ("out_planes", ctypes.c_void_p),
         ("lse_planes", ctypes.c_void_p),
         ("t_c", ctypes.c_int32 * (AS_MAX_P * AS_MAX_P)),
+        ("g", ctypes.c_int), ("n_groups", ctypes.c_int),
+        ("member", ctypes.c_uint64 * (AS_MAX_P * AS_MAX_P)),
     ]
 
 
@@ -76,6 +79,11 @@ def _load() -> ctypes.CDLL:
     lib.as_cache_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int]
     lib.as_cache_init.restype = c_int
     lib.as_cache_init.argtypes = [ctypes.POINTER(AsCacheStruct), vp, sz, c_int, c_int, c_int, c_int, c_int, c_int]
+    lib.as_cache_group_bytes.restype = sz
+    lib.as_cache_group_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int, c_int]
+    lib.as_cache_group_init.restype = c_int
+    lib.as_cache_group_init.argtypes = [ctypes.POINTER(AsCacheStruct), vp, sz, c_int, c_int, c_int, c_int, c_int,
+                                        c_int, c_int]
     lib.as_plan_resolve.restype = c_int
     lib.as_plan_resolve.argtypes = [ctypes.POINTER(AsCacheStruct), vp, c_int, vp, vp]
     lib.as_step.restype = c_int

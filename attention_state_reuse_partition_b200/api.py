@@ -77,58 +77,93 @@ def as_compose(outs, lses, out=None, lse=None, stream=None):
     return out, lse
 
 
-def as_cache_bytes(B: int, H: int, S: int, d: int, P: int) -> int:
-    return int(LIB.as_cache_bytes(B, H, S, d, P, AS_F32))
+def _cache_dt(cache_dtype) -> int:
+    if cache_dtype in (torch.float32, "f32", AS_F32):
+        return AS_F32
+    if cache_dtype in (torch.bfloat16, "bf16", AS_BF16):
+        return AS_BF16
+    raise AsError(_lib.AS_ERR_INVALID_ARG, f"unsupported cache dtype {cache_dtype}")
+
+
+def as_cache_bytes(B: int, H: int, S: int, d: int, P: int, g: int = 1, cache_dtype=torch.float32) -> int:
+    return int(LIB.as_cache_group_bytes(B, H, S, d, P, g, _cache_dt(cache_dtype)))
 
 
 class AsCache:
-    """A state cache: the C struct plus its device buffer (allocated with torch)."""
+    """A state cache: the C struct plus its device buffer (allocated with
+    torch).  ``g``: KV partitions per cache group (one composed entry per
+    (query partition, group)); ``cache_dtype``: torch.float32 or
+    torch.bfloat16 for the OUT entries (LSE entries are fp32)."""
 
-    def __init__(self, B: int, H: int, S: int, d: int, P: int, device="cuda", buffer: Optional[torch.Tensor] = None):
-        nbytes = as_cache_bytes(B, H, S, d, P)
+    def __init__(self, B: int, H: int, S: int, d: int, P: int, device="cuda", buffer: Optional[torch.Tensor] = None,
+                 g: int = 1, cache_dtype=torch.float32):
+        dt = _cache_dt(cache_dtype)
+        nbytes = as_cache_bytes(B, H, S, d, P, g, dt)
         if nbytes == 0:
             raise AsError(_lib.AS_ERR_INVALID_ARG, "invalid cache sizes")
         if buffer is None:
             buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.buffer = buffer
         self.struct = AsCacheStruct()
-        check(LIB.as_cache_init(ctypes.byref(self.struct), buffer.data_ptr(), buffer.numel(), B, H, S, d, P, AS_F32))
-        self.B, self.H, self.S, self.d, self.P = B, H, S, d, P
+        check(LIB.as_cache_group_init(ctypes.byref(self.struct), buffer.data_ptr(), buffer.numel(), B, H, S, d, P, g,
+                                      dt))
+        self._set_sizes(B, H, S, d, P, g, dt)
+
+    def _set_sizes(self, B, H, S, d, P, g, dt):
+        self.B, self.H, self.S, self.d, self.P, self.g = B, H, S, d, P, g
+        self.NG = (P + g - 1) // g
+        self.cache_dtype = torch.bfloat16 if dt == AS_BF16 else torch.float32
 
     @classmethod
-    def host_only(cls, B: int, H: int, S: int, d: int, P: int) -> "AsCache":
+    def host_only(cls, B: int, H: int, S: int, d: int, P: int, g: int = 1, cache_dtype=torch.float32) -> "AsCache":
         """A cache struct for host-side plan bookkeeping (as_plan_resolve) on a
         machine without a GPU.  Its planes point at a placeholder address that
         is never dereferenced; it must not be passed to as_step."""
         self = cls.__new__(cls)
         self.buffer = None
         self.struct = AsCacheStruct()
-        check(LIB.as_cache_init(ctypes.byref(self.struct), 1 << 30, as_cache_bytes(B, H, S, d, P),
-                                B, H, S, d, P, AS_F32))
-        self.B, self.H, self.S, self.d, self.P = B, H, S, d, P
+        dt = _cache_dt(cache_dtype)
+        check(LIB.as_cache_group_init(ctypes.byref(self.struct), 1 << 30, as_cache_bytes(B, H, S, d, P, g, dt),
+                                      B, H, S, d, P, g, dt))
+        self._set_sizes(B, H, S, d, P, g, dt)
         return self
 
     def set_t_c(self, t_c) -> None:
-        """Overwrite the host-side store timestamps (for replaying bookkeeping)."""
+        """Overwrite the host-side store timestamps [P, n_groups] (for
+        replaying bookkeeping)."""
         flat = np.asarray(t_c, dtype=np.int32).reshape(-1)
-        for x in range(self.P * self.P):
+        for x in range(self.P * self.NG):
             self.struct.t_c[x] = int(flat[x])
+
+    def set_member(self, member) -> None:
+        """Overwrite the stored member masks [P, n_groups] (bit j = KV
+        partition j), for replaying bookkeeping."""
+        flat = np.asarray(member, dtype=np.uint64).reshape(-1)
+        for x in range(self.P * self.NG):
+            self.struct.member[x] = int(flat[x])
 
     @property
     def t_c(self) -> np.ndarray:
-        return np.ctypeslib.as_array(self.struct.t_c)[: self.P * self.P].reshape(self.P, self.P).copy()
+        return np.ctypeslib.as_array(self.struct.t_c)[: self.P * self.NG].reshape(self.P, self.NG).copy()
+
+    @property
+    def member(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.struct.member)[: self.P * self.NG].reshape(self.P, self.NG).copy()
 
     def planes(self):
-        """Views of the cache planes: OUT [P,B,H,S,d], LSE [P,B,H,S] (fp32)."""
-        n_out = self.P * self.B * self.H * self.S * self.d
-        n_lse = self.P * self.B * self.H * self.S
-        f = self.buffer.view(torch.float32)
-        return (f[:n_out].view(self.P, self.B, self.H, self.S, self.d),
-                f[n_out:n_out + n_lse].view(self.P, self.B, self.H, self.S))
+        """Views of the cache planes: OUT [NG,B,H,S,d] (the cache dtype), LSE
+        [NG,B,H,S] (fp32)."""
+        n_out = self.NG * self.B * self.H * self.S * self.d
+        n_lse = self.NG * self.B * self.H * self.S
+        esz = 2 if self.cache_dtype == torch.bfloat16 else 4
+        out = self.buffer[: n_out * esz].view(self.cache_dtype).view(self.NG, self.B, self.H, self.S, self.d)
+        lse = self.buffer[n_out * esz: n_out * esz + n_lse * 4].view(torch.float32).view(
+            self.NG, self.B, self.H, self.S)
+        return out, lse
 
 
-def as_cache_init(B, H, S, d, P, device="cuda", buffer=None) -> AsCache:
-    return AsCache(B, H, S, d, P, device=device, buffer=buffer)
+def as_cache_init(B, H, S, d, P, device="cuda", buffer=None, g: int = 1, cache_dtype=torch.float32) -> AsCache:
+    return AsCache(B, H, S, d, P, device=device, buffer=buffer, g=g, cache_dtype=cache_dtype)
 
 
 def _plan_bytes(plan, P):

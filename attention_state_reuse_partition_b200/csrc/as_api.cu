@@ -89,20 +89,39 @@ void base_launch(asp::AttnLaunch& L, const void* q, const void* k, const void* v
   L.poll_budget = 1u << 24;
 }
 
-// hit / age of a plan against cache timestamps; codes checked first, then misses
+// bit mask of the members of group (i, G) that carry plan code `code`
+uint64_t group_mask(const uint8_t* plan, int P, int g, int i, int G, uint8_t code) {
+  uint64_t m = 0;
+  for (int j = G * g; j < std::min((G + 1) * g, P); ++j)
+    if (plan[i * P + j] == code) m |= uint64_t(1) << j;
+  return m;
+}
+
+// hit / age of a plan against the cache bookkeeping; codes checked first, then
+// groups that mix reuse and store, then misses (never stored, or other members)
 as_status resolve(const as_cache* c, const uint8_t* plan, int step, uint8_t* hit, int32_t* age) {
-  const int P = c->P;
+  const int P = c->P, g = c->g, NG = c->n_groups;
   for (int x = 0; x < P * P; ++x)
     if (plan[x] > AS_PLAN_FRESH_STORE)
       return fail(AS_ERR_INVALID_ARG, "plan[%d][%d] = %d is not 0, 1 or 2", x / P, x % P, plan[x]);
-  for (int x = 0; x < P * P; ++x) {
-    if (plan[x] == AS_PLAN_REUSE && c->t_c[x] < 0)
-      return fail(AS_ERR_CACHE_MISS, "pair (%d, %d) is reused but its cache entry was never stored", x / P, x % P);
-  }
+  for (int i = 0; i < P; ++i)
+    for (int G = 0; G < NG; ++G)
+      if (group_mask(plan, P, g, i, G, AS_PLAN_REUSE) && group_mask(plan, P, g, i, G, AS_PLAN_FRESH_STORE))
+        return fail(AS_ERR_INVALID_ARG, "group (%d, %d) of size %d both reuses and stores members", i, G, g);
+  for (int i = 0; i < P; ++i)
+    for (int G = 0; G < NG; ++G) {
+      const uint64_t r = group_mask(plan, P, g, i, G, AS_PLAN_REUSE);
+      if (!r) continue;
+      if (c->t_c[i * NG + G] < 0)
+        return fail(AS_ERR_CACHE_MISS, "group (%d, %d) is reused but its cache entry was never stored", i, G);
+      if (r != c->member[i * NG + G])
+        return fail(AS_ERR_CACHE_MISS, "group (%d, %d) reuses members 0x%llx but stores 0x%llx", i, G,
+                    static_cast<unsigned long long>(r), static_cast<unsigned long long>(c->member[i * NG + G]));
+    }
   for (int x = 0; x < P * P; ++x) {
     const bool r = plan[x] == AS_PLAN_REUSE;
     if (hit) hit[x] = r ? 1 : 0;
-    if (age) age[x] = r ? step - c->t_c[x] : 0;
+    if (age) age[x] = r ? step - c->t_c[(x / P) * NG + (x % P) / g] : 0;
   }
   return AS_OK;
 }
@@ -245,18 +264,27 @@ as_status as_compose(const float* outs, const float* lses, int n_states, int64_t
   return ok();
 }
 
-size_t as_cache_bytes(int B, int H, int S, int d, int P, as_dtype cache_dt) {
-  if (cache_dt != AS_F32) return 0;
-  if (check_shape(B, H, S, d, P) != AS_OK) return 0;
-  return static_cast<size_t>(P) * B * H * S * (d + 1) * sizeof(float);
+size_t as_cache_group_bytes(int B, int H, int S, int d, int P, int g, as_dtype cache_dt) {
+  if (cache_dt != AS_F32 && cache_dt != AS_BF16) return 0;
+  if (check_shape(B, H, S, d, P) != AS_OK || g < 1 || g > P) return 0;
+  const size_t NG = static_cast<size_t>((P + g - 1) / g);
+  const size_t rows = static_cast<size_t>(B) * H * S;
+  return NG * rows * (static_cast<size_t>(d) * (cache_dt == AS_BF16 ? 2 : 4) + sizeof(float));
 }
 
-as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, as_dtype cache_dt) {
+size_t as_cache_bytes(int B, int H, int S, int d, int P, as_dtype cache_dt) {
+  return as_cache_group_bytes(B, H, S, d, P, 1, cache_dt);
+}
+
+as_status as_cache_group_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, int g,
+                              as_dtype cache_dt) {
   if (!c) return fail(AS_ERR_INVALID_ARG, "null cache struct");
-  if (cache_dt != AS_F32) return fail(AS_ERR_UNSUPPORTED, "only fp32 cache entries are built");
+  if (cache_dt != AS_F32 && cache_dt != AS_BF16)
+    return fail(AS_ERR_INVALID_ARG, "cache dtype %d is not AS_F32 or AS_BF16", static_cast<int>(cache_dt));
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
-  const size_t need = as_cache_bytes(B, H, S, d, P, cache_dt);
+  if (g < 1 || g > P) return fail(AS_ERR_INVALID_ARG, "group size %d outside [1, %d]", g, P);
+  const size_t need = as_cache_group_bytes(B, H, S, d, P, g, cache_dt);
   if (!buf || (reinterpret_cast<uintptr_t>(buf) & 255u) != 0)
     return fail(AS_ERR_INVALID_ARG, "cache buffer must be non-null and 256-byte aligned");
   if (bytes < need) return fail(AS_ERR_INVALID_ARG, "cache buffer has %zu bytes, needs %zu", bytes, need);
@@ -267,11 +295,18 @@ as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int 
   c->S = S;
   c->d = d;
   c->P = P;
+  c->g = g;
+  c->n_groups = (P + g - 1) / g;
   c->cache_dt = cache_dt;
-  c->out_planes = static_cast<float*>(buf);
-  c->lse_planes = c->out_planes + static_cast<size_t>(P) * B * H * S * d;
+  c->out_planes = buf;
+  const size_t out_bytes = static_cast<size_t>(c->n_groups) * B * H * S * d * (cache_dt == AS_BF16 ? 2 : 4);
+  c->lse_planes = reinterpret_cast<float*>(static_cast<char*>(buf) + out_bytes);
   for (int x = 0; x < AS_MAX_P * AS_MAX_P; ++x) c->t_c[x] = -1;
   return ok();
+}
+
+as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, as_dtype cache_dt) {
+  return as_cache_group_init(c, buf, bytes, B, H, S, d, P, 1, cache_dt);
 }
 
 as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step, uint8_t* h_hit, int32_t* h_age) {
@@ -292,15 +327,15 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(AS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   if (!(scale > 0.f)) return fail(AS_ERR_INVALID_ARG, "scale must be > 0");
-  const int B = c->B, H = c->H, S = c->S, d = c->d, P = c->P, n = S / P;
+  const int B = c->B, H = c->H, S = c->S, d = c->d, P = c->P, n = S / P, g = c->g, NG = c->n_groups;
   uint8_t hit[AS_MAX_P * AS_MAX_P];
   int32_t age[AS_MAX_P * AS_MAX_P];
   if ((s = resolve(c, h_plan, step, hit, age)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // fresh pairs: composite of the plain-fresh partitions -> out/lse, stored
-  // pairs -> their cache planes
+  // fresh pairs: composite of the plain-fresh partitions -> out/lse; the
+  // stored members of each group -> one composed state in the group's plane
   asp::AttnLaunch L;
   base_launch(L, q, k, v, B, H, S, d, P, scale);
   L.n_blocks = P;
@@ -316,7 +351,7 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
       need_compose |= pc != AS_PLAN_FRESH;
     }
   }
-  for (int j = 0; j < P; ++j) L.dest_of[j] = static_cast<int8_t>(j);
+  for (int j = 0; j < P; ++j) L.dest_of[j] = static_cast<int8_t>(j / g);
   // every query partition reads the same KV list: one block of S rows, so
   // query tiles are not cut at partition boundaries
   bool uniform = true;
@@ -330,6 +365,7 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   L.out_rows = S;
   L.out_row0 = 0;
   L.dst_out = c->out_planes;
+  L.dst_bf16 = c->cache_dt == AS_BF16;
   L.dst_lse = c->lse_planes;
   L.dst_rows = S;
   L.dst_row0 = 0;
@@ -337,7 +373,7 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   L.dst_plane_lse = static_cast<long long>(B) * H * S;
   if (any_fresh && (s = launch_attn(L, dt, st)) != AS_OK) return s;
 
-  // final composition: composite + stored fresh states + reused entries
+  // final composition: composite + stored group entries + reused group entries
   if (need_compose) {
     asp::ComposePlan a;
     std::memset(&a, 0, sizeof(a));
@@ -359,11 +395,13 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
         continue;
       }
       if (has_fresh) a.src[i][cnt++] = -1;
-      for (int j = 0; j < P; ++j)
-        if (h_plan[i * P + j] != AS_PLAN_FRESH) a.src[i][cnt++] = static_cast<int8_t>(j);
+      for (int G = 0; G < NG; ++G)
+        if (group_mask(h_plan, P, g, i, G, AS_PLAN_REUSE) || group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE))
+          a.src[i][cnt++] = static_cast<int8_t>(G);
       a.nsrc[i] = static_cast<uint8_t>(cnt);
     }
     a.cache_out = c->out_planes;
+    a.cache_bf16 = c->cache_dt == AS_BF16;
     a.cache_lse = c->lse_planes;
     a.plane_out = L.dst_plane_out;
     a.plane_lse = L.dst_plane_lse;
@@ -373,8 +411,13 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
     if (e != cudaSuccess) return cuda_fail(e, "step compose launch");
   }
 
-  for (int x = 0; x < P * P; ++x)
-    if (h_plan[x] == AS_PLAN_FRESH_STORE) c->t_c[x] = step;
+  for (int i = 0; i < P; ++i)
+    for (int G = 0; G < NG; ++G) {
+      const uint64_t m = group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE);
+      if (!m) continue;
+      c->t_c[i * NG + G] = step;
+      c->member[i * NG + G] = m;
+    }
   if (h_hit) std::memcpy(h_hit, hit, static_cast<size_t>(P) * P);
   if (h_age) std::memcpy(h_age, age, static_cast<size_t>(P) * P * sizeof(int32_t));
   return ok();
@@ -555,6 +598,8 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
   if ((s = check_cache(c)) != AS_OK) return s;
   const int P = pl->P;
   if (c->P != P) return fail(AS_ERR_INVALID_ARG, "cache and planner disagree on P");
+  if (c->g != 1 || c->cache_dt != AS_F32)
+    return fail(AS_ERR_UNSUPPORTED, "the anchor statistics read per-pair fp32 entries: the cache needs g = 1 and AS_F32");
   if (!lse_full || !local_anchor || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
   const int B = c->B, H = c->H, S = c->S, d = c->d, n = S / P;
   if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
@@ -567,7 +612,7 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
       sel.v[i * P + j] = (h_plan[i * P + j] == AS_PLAN_FRESH_STORE && std::abs(i - j) > pl->window) ? 1 : 0;
   double* partials = static_cast<double*>(scratch);
   double* sums = partials + static_cast<size_t>(P) * P * B * H * 2;
-  cudaError_t e = asp::launch_anchor_stats(c->out_planes, c->lse_planes, lse_full,
+  cudaError_t e = asp::launch_anchor_stats(static_cast<const float*>(c->out_planes), c->lse_planes, lse_full,
                                            static_cast<long long>(B) * H * S * d, static_cast<long long>(B) * H * S,
                                            P, B * H, S, d, sel, partials, sums, st);
   if (e != cudaSuccess) return cuda_fail(e, "anchor statistics launch");

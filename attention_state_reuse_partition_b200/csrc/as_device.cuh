@@ -7,6 +7,7 @@
 // flag and returns as well, so the CTA drains and exits instead of hanging.
 #pragma once
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "as_kernels.h"
@@ -327,8 +328,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------------------
 // A query row block reads a list of KV token ranges grouped into accumulation
 // groups.  Group 0 (when present) gathers every code-1 partition (adjacent
-// partitions merged into one range) and is emitted as one composed state; each
-// code-2 partition forms its own group, emitted as that partition's state.
+// partitions merged into one range) and is emitted as one composed state.
+// Consecutive code-2 partitions with the same destination plane form one
+// group, emitted as the composed state of its partitions (a cache group entry;
+// with one destination per partition, each partition's own state).
 struct KvSchedule {
   int n_ranges;
   int n_groups;
@@ -361,11 +364,24 @@ __device__ __forceinline__ void build_schedule(const uint8_t* code_row, const in
   }
   for (int j = 0; j < P; ++j) {
     if (code_row[j] != AS_KCODE_EMIT) continue;
+    const int dst = dest_of[j];
+    if (s.n_groups > 0 && s.group_dest[s.n_groups - 1] == dst) {
+      // same destination as the previous emitted partition: one group
+      if (s.range_hi[s.n_ranges - 1] == j * n) {
+        s.range_hi[s.n_ranges - 1] = (j + 1) * n;
+      } else {
+        s.range_lo[s.n_ranges] = j * n;
+        s.range_hi[s.n_ranges] = (j + 1) * n;
+        ++s.n_ranges;
+        ++s.group_count[s.n_groups - 1];
+      }
+      continue;
+    }
     s.range_lo[s.n_ranges] = j * n;
     s.range_hi[s.n_ranges] = (j + 1) * n;
     s.group_first[s.n_groups] = s.n_ranges;
     s.group_count[s.n_groups] = 1;
-    s.group_dest[s.n_groups] = dest_of[j];
+    s.group_dest[s.n_groups] = dst;
     ++s.n_ranges;
     ++s.n_groups;
   }

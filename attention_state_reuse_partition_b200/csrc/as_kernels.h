@@ -29,14 +29,18 @@ struct AttnLaunch {
   // uses row b of `code` ([n_blocks][P])
   int n_blocks, block_rows, block_row0;
   uint8_t code[AS_MAX_P * AS_MAX_P];
-  int8_t dest_of[AS_MAX_P];  // destination plane of each AS_KCODE_EMIT partition
+  // destination plane of each AS_KCODE_EMIT partition; consecutive emitted
+  // partitions with the same destination form one accumulation group
+  int8_t dest_of[AS_MAX_P];
   // composite output: row s of head bh at ((bh * out_rows) + s - out_row0)
   float* out;
   float* lse;
   int out_rows, out_row0;
-  // emitted planes: plane p, row s of head bh at p * plane + (bh * dst_rows + s - dst_row0)
-  float* dst_out;
+  // emitted planes: plane p, row s of head bh at p * plane + (bh * dst_rows + s - dst_row0);
+  // OUT in fp32, or in bf16 (round to nearest even) when dst_bf16
+  void* dst_out;
   float* dst_lse;
+  int dst_bf16;
   int dst_rows, dst_row0;
   long long dst_plane_out, dst_plane_lse;
   unsigned int poll_budget;
@@ -57,9 +61,10 @@ struct ComposeStrided {
 // query partition from the step plan
 struct ComposePlan {
   int B, H, S, d, P, n;
-  int8_t src[AS_MAX_P][AS_MAX_P + 1];  // per query partition: -1 = composite, j = cache plane j
+  int8_t src[AS_MAX_P][AS_MAX_P + 1];  // per query partition: -1 = composite, G = cache plane G
   uint8_t nsrc[AS_MAX_P];
-  const float* cache_out;
+  const void* cache_out;  // fp32, or bf16 when cache_bf16
+  int cache_bf16;
   const float* cache_lse;
   long long plane_out, plane_lse;
   float* out;  // [B,H,S,d]: holds the composite on entry (where used), the final state on exit

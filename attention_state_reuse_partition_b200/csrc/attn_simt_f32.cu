@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(ROWS) attn_simt_kernel(const __grid_constant__
     if (s_row < q_hi) {
       const int dest = sched.group_dest[g];
       float* orow;
+      __nv_bfloat16* brow = nullptr;  // bf16 cache planes
       float* lrow;
       if (dest < 0) {
         const long long r_idx = static_cast<long long>(bh) * L.out_rows + (s_row - L.out_row0);
@@ -96,12 +97,19 @@ __global__ void __launch_bounds__(ROWS) attn_simt_kernel(const __grid_constant__
         lrow = L.lse + r_idx;
       } else {
         const long long r_idx = static_cast<long long>(bh) * L.dst_rows + (s_row - L.dst_row0);
-        orow = L.dst_out + dest * L.dst_plane_out + r_idx * D;
+        const long long e_idx = dest * L.dst_plane_out + r_idx * D;
+        orow = static_cast<float*>(L.dst_out) + e_idx;
+        if (L.dst_bf16) brow = static_cast<__nv_bfloat16*>(L.dst_out) + e_idx;
         lrow = L.dst_lse + dest * L.dst_plane_lse + r_idx;
       }
       const float inv_l = 1.0f / l;
+      if (brow) {
 #pragma unroll
-      for (int e = 0; e < D; ++e) orow[e] = o[e] * inv_l;
+        for (int e = 0; e < D; ++e) brow[e] = __float2bfloat16_rn(o[e] * inv_l);
+      } else {
+#pragma unroll
+        for (int e = 0; e < D; ++e) orow[e] = o[e] * inv_l;
+      }
       *lrow = m + logf(l);
     }
   }

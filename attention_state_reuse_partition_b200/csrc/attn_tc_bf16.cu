@@ -443,7 +443,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // the warp's 32 rows are consecutive in the destination: s_row0 + rr
         const int s_row0 = s_row - lane;
         const int dest = c.sched.group_dest[group];
-        float* orow0;  // row s_row0
+        float* orow0;  // row s_row0 (fp32 destinations)
+        __nv_bfloat16* brow0 = nullptr;  // row s_row0 (bf16 cache planes)
         float* lrow;
         if (dest < 0) {
           const long long r_idx = static_cast<long long>(bh) * L.out_rows + (s_row0 - L.out_row0);
@@ -451,7 +452,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           lrow = L.lse + r_idx + lane;
         } else {
           const long long r_idx = static_cast<long long>(bh) * L.dst_rows + (s_row0 - L.dst_row0);
-          orow0 = L.dst_out + dest * L.dst_plane_out + r_idx * D;
+          const long long e_idx = dest * L.dst_plane_out + r_idx * D;
+          orow0 = static_cast<float*>(L.dst_out) + e_idx;
+          if (L.dst_bf16) brow0 = static_cast<__nv_bfloat16*>(L.dst_out) + e_idx;
           lrow = L.dst_lse + dest * L.dst_plane_lse + r_idx + lane;
         }
         const float inv_l = 1.0f / l;
@@ -478,8 +481,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int i = 0; i < 4; ++i) {
             const int rr = 8 * i + rb_row;
             const float4 v4 = *reinterpret_cast<const float4*>(stage + rr * STAGE_LD + rb_col);
-            if (s_row0 + rr < q_hi)
-              *reinterpret_cast<float4*>(orow0 + static_cast<long long>(rr) * D + ch * 16 + rb_col) = v4;
+            const long long off = static_cast<long long>(rr) * D + ch * 16 + rb_col;
+            if (s_row0 + rr < q_hi) {
+              if (brow0)
+                *reinterpret_cast<uint2*>(brow0 + off) = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
+              else
+                *reinterpret_cast<float4*>(orow0 + off) = v4;
+            }
           }
           __syncwarp();
         }

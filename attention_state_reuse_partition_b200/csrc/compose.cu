@@ -24,10 +24,22 @@ constexpr int SM_COUNT = 148;
 
 template <int D>
 struct Vec;
+// a packed pair of bf16 (low half = first element) widened to fp32
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
 template <>
 struct Vec<128> {
   using T = float4;
   static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  // this lane's 4 elements of row `row` of a fp32 or bf16 state
+  static __device__ __forceinline__ float4 load(const void* base, long long row, int lane, bool bf16) {
+    if (bf16) {
+      const uint2 u = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + row * 128)[lane];
+      return make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
+    }
+    return reinterpret_cast<const float4*>(static_cast<const float*>(base) + row * 128)[lane];
+  }
   static __device__ __forceinline__ void fma(float4& a, float c, const float4& x) {
     a.x = fmaf(c, x.x, a.x);
     a.y = fmaf(c, x.y, a.y);
@@ -39,6 +51,13 @@ template <>
 struct Vec<64> {
   using T = float2;
   static __device__ __forceinline__ float2 zero() { return make_float2(0.f, 0.f); }
+  static __device__ __forceinline__ float2 load(const void* base, long long row, int lane, bool bf16) {
+    if (bf16) {
+      const uint32_t u = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(base) + row * 64)[lane];
+      return make_float2(bf_lo(u), bf_hi(u));
+    }
+    return reinterpret_cast<const float2*>(static_cast<const float*>(base) + row * 64)[lane];
+  }
   static __device__ __forceinline__ void fma(float2& a, float c, const float2& x) {
     a.x = fmaf(c, x.x, a.x);
     a.y = fmaf(c, x.y, a.y);
@@ -56,9 +75,15 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+struct Ptrs {
+  const void* first;    // OUT base
+  const float* second;  // LSE base
+  bool bf16;            // OUT in bf16
+};
+
 // Composes rows [row0, row0+nr) (nr <= RB) of `nsrc` sources.  src(k) gives the
 // base pointers (out_base, lse_base) of source k such that row r's state is at
-// out_base + r*D and lse_base + r.  The output may alias a source: every source
+// row r of out_base (fp32, or bf16 when the source says so) and lse_base + r.  The output may alias a source: every source
 // row is read before the output row is written, by the same warp.
 template <int D, class SrcFn>
 __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, SrcFn src, float* out,
@@ -117,13 +142,16 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, S
       for (; kk + 8 <= kn; kk += 8) {
         T x[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          x[u] = reinterpret_cast<const T*>(src(k0 + kk + u).first + (row0 + rr) * D)[lane];
+        for (int u = 0; u < 8; ++u) {
+          const Ptrs sp = src(k0 + kk + u);
+          x[u] = V::load(sp.first, row0 + rr, lane, sp.bf16);
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u) V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk + u), x[u]);
       }
       for (; kk < kn; ++kk) {
-        const T x = reinterpret_cast<const T*>(src(k0 + kk).first + (row0 + rr) * D)[lane];
+        const Ptrs sp = src(k0 + kk);
+        const T x = V::load(sp.first, row0 + rr, lane, sp.bf16);
         V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk), x);
       }
     }
@@ -136,11 +164,6 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, S
   }
 }
 
-struct Ptrs {
-  const float* first;
-  const float* second;
-};
-
 template <int D>
 __global__ void __launch_bounds__(WARPS * 32) compose_strided_kernel(const __grid_constant__ ComposeStrided a) {
   const int lane = threadIdx.x & 31;
@@ -148,7 +171,7 @@ __global__ void __launch_bounds__(WARPS * 32) compose_strided_kernel(const __gri
   const long long gw = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
   const long long stride = static_cast<long long>(gridDim.x) * WARPS;
   auto src = [&](int k) {
-    return Ptrs{a.outs + k * a.stride_out, a.lses + k * a.stride_lse};
+    return Ptrs{a.outs + k * a.stride_out, a.lses + k * a.stride_lse, false};
   };
   for (long long b = gw; b < nblk; b += stride) {
     const long long row0 = b * RB;
@@ -175,8 +198,10 @@ __global__ void __launch_bounds__(WARPS * 32) compose_plan_kernel(const __grid_c
     const int8_t* list = a.src[i];
     auto src = [&](int k) {
       const int j = list[k];
-      if (j < 0) return Ptrs{a.out, a.lse};
-      return Ptrs{a.cache_out + j * a.plane_out, a.cache_lse + j * a.plane_lse};
+      if (j < 0) return Ptrs{a.out, a.lse, false};
+      if (a.cache_bf16)
+        return Ptrs{static_cast<const __nv_bfloat16*>(a.cache_out) + j * a.plane_out, a.cache_lse + j * a.plane_lse, true};
+      return Ptrs{static_cast<const float*>(a.cache_out) + j * a.plane_out, a.cache_lse + j * a.plane_lse, false};
     };
     compose_rows<D>(row0, nr, a.nsrc[i], src, a.out, a.lse, lane);
   }

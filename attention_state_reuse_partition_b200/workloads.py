@@ -225,6 +225,28 @@ def plan_for_step(s: Spec, t: int):
     return plan
 
 
+def grouped_plan_for_step(s: Spec, t: int, g: int):
+    """plan_for_step for a cache of groups of g KV partitions (group j // g).
+
+    A group is stored or reused as a whole, so the per-pair plan is lifted to
+    groups: for query partition i and group G, the members outside the window
+    are stored if the pair plan stores any of them (the anchor, or a forced
+    pair), else reused; members inside the window stay fresh.
+    """
+    base = plan_for_step(s, t)
+    plan = base.clone()
+    P = s.P
+    for i in range(P):
+        for G in range((P + g - 1) // g):
+            js = [j for j in range(G * g, min((G + 1) * g, P)) if base[i, j] != PLAN_FRESH]
+            if not js:
+                continue
+            code = PLAN_FRESH_STORE if any(base[i, j] == PLAN_FRESH_STORE for j in js) else PLAN_REUSE
+            for j in js:
+                plan[i, j] = code
+    return plan
+
+
 def all_fresh_plan(P: int):
     return torch.full((P, P), PLAN_FRESH, dtype=torch.uint8)
 

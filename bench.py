@@ -375,18 +375,24 @@ def run_reuse(args, device):
             "reuse_mse_vs_full": mse}
 
 
-def run_video_long(args, device):
+def run_video_long(args, device, g=1, cache_dtype="f32"):
     """Long video trajectory: an anchor step, then three reuse steps (window 4,
-    a seeded 10% of reused pairs forced fresh and stored each step)."""
+    a seeded 10% of reused pairs forced fresh and stored each step).  With
+    g > 1 the cache keeps one composed entry per (query partition, group of g
+    KV partitions) and a forced pair refreshes its whole group."""
     from attention_state_reuse_partition_b200 import api
     s = W.spec("video_long")
-    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, g=g, cache_dtype=cache_dtype)
+    NG = (s.P + g - 1) // g
+    entry_bytes = s.B * s.H * s.n * (s.d * (2 if cache_dtype == "bf16" else 4) + 4)  # one (i, G) entry
     out = torch.empty((s.B, s.H, s.S, s.d), device=device)
     lse = torch.empty((s.B, s.H, s.S), device=device)
     per_step = []
     last = None
     for t, q, k, v in W.video_trajectory(s, device=device):
-        plan = W.plan_for_step(s, t).numpy()
+        plan = W.grouped_plan_for_step(s, t, g).numpy()
+        reused_entries = sum(bool((plan[i, G * g:(G + 1) * g] == W.PLAN_REUSE).any())
+                             for i in range(s.P) for G in range(NG))
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         api.as_step(cache, q, k, v, plan, t, out=out, lse=lse)
@@ -398,15 +404,21 @@ def run_video_long(args, device):
         ms = a.elapsed_time(b)
         fl = 4.0 * s.B * s.H * n_fresh * s.n * s.n * s.d
         per_step.append({"step": t, "ms": round(ms, 3), "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
-                         "stored_pairs": n_store, "fresh_tflops_whole_step": round(fl / (ms * 1e-3) / 1e12, 1)})
+                         "stored_pairs": n_store, "reused_entries": reused_entries,
+                         "reuse_read_gb": round(reused_entries * entry_bytes / 1e9, 3),
+                         "fresh_tflops_whole_step": round(fl / (ms * 1e-3) / 1e12, 1)})
         last = (q, k, v)
     q, k, v = last
     full_o, _ = api.as_partition_attn(q, k, v, s.P, -1, list(range(s.P)))
     torch.cuda.synchronize()
     mse = torch.mean((out - full_o) ** 2).item()
+    cache_gb = cache.buffer.numel() / 1e9
     del cache, full_o, out, lse, last, q, k, v
     torch.cuda.empty_cache()
-    return {"workload": "video_long (4 steps)", "steps": per_step, "reuse_mse_vs_full_last_step": mse}
+    name = "video_long (4 steps)" if g == 1 and cache_dtype == "f32" else \
+        f"video_long (4 steps), cache groups of {g} partitions, {cache_dtype} OUT entries"
+    return {"workload": name, "g": g, "cache_dtype": cache_dtype, "cache_gb": round(cache_gb, 2),
+            "steps": per_step, "reuse_mse_vs_full_last_step": mse}
 
 
 def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5):
@@ -461,7 +473,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
-    ap.add_argument("--only", choices=["compose", "reuse", "video_long", "planner"], default=None,
+    ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
@@ -481,6 +493,7 @@ def main():
     device = torch.device("cuda", local)
     if args.only is not None:
         fn = {"compose": run_compose, "reuse": run_reuse, "video_long": run_video_long,
+              "video_long_grouped": lambda a, dev: run_video_long(a, dev, g=4, cache_dtype="bf16"),
               "planner": run_planner}[args.only]
         print(json.dumps({"only": args.only, **fn(args, device)}))
         return
@@ -499,6 +512,7 @@ def main():
         secondary["compose"] = comp
         secondary["reuse"] = run_reuse(args, device)
         secondary["video_long"] = run_video_long(args, device)
+        secondary["video_long_grouped"] = run_video_long(args, device, g=4, cache_dtype="bf16")
         secondary["planner"] = run_planner(args, device)
 
     cpu = None

@@ -45,7 +45,7 @@ typedef enum {
   AS_OK = 0,
   AS_ERR_INVALID_ARG = 1,  /* shapes, alignment, plan values, cache mismatch */
   AS_ERR_UNSUPPORTED = 2,  /* valid request outside the built paths */
-  AS_ERR_CACHE_MISS = 3,   /* the plan reuses a pair whose entry was never stored */
+  AS_ERR_CACHE_MISS = 3,   /* the plan reuses an entry never stored, or other members than stored */
   AS_ERR_CUDA = 4,         /* a CUDA runtime call failed (message in as_last_error) */
   AS_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see as_device_status) */
 } as_status;
@@ -95,43 +95,77 @@ as_status as_compose(const float* outs, const float* lses, int n_states, int64_t
                      int64_t state_stride_out, int64_t state_stride_lse,
                      float* out, float* lse, void* stream);
 
-/* State cache: one entry per (query partition i, KV partition j), stored as
- * P planes [P][B,H,S,d] (OUT) and [P][B,H,S] (LSE) in a caller-owned device
- * buffer; entry (i, j) is plane j at the rows of partition i.  The host-side
- * t_c[i*P+j] is the step of the entry's last store (-1 = never stored).
- * The struct is caller-owned host memory; initialise it with as_cache_init. */
+/* State cache.  KV partitions are merged into groups of g consecutive
+ * partitions (group G = {j : j / g = G}, n_groups = ceil(P / g); the last
+ * group may be short), following DiTango's memory-aware state merging
+ * (review page, "If this is right", second bullet: composed states "can be
+ * merged into coarser groups under memory pressure"; Axiom & Free-Parameter
+ * Ledger: group size g = 4/8/16).  The cache holds one composed state per
+ * (query partition i, group G): the composition of the states of the members
+ * stored at its last refresh.  g = 1 gives one entry per (i, j) pair.
+ *
+ * Storage, in one caller-owned device buffer: OUT planes [n_groups][B,H,S,d]
+ * (fp32, or bf16 rounded to nearest even when cache_dt = AS_BF16), then LSE
+ * planes [n_groups][B,H,S] (fp32 always); entry (i, G) is plane G at the rows
+ * of partition i.  Host side: t_c[i*n_groups+G] is the step of the entry's
+ * last store (-1 = never stored) and member[i*n_groups+G] the bit mask (bit
+ * j) of the KV partitions it was composed from.  The struct is caller-owned
+ * host memory; initialise it with as_cache_init or as_cache_group_init. */
 typedef struct as_cache {
   uint32_t magic;
   int B, H, S, d, P;
-  as_dtype cache_dt;
-  float* out_planes;  /* device, [P][B,H,S,d] */
-  float* lse_planes;  /* device, [P][B,H,S] */
+  as_dtype cache_dt;  /* type of the OUT planes: AS_F32 or AS_BF16 */
+  void* out_planes;   /* device, [n_groups][B,H,S,d] of cache_dt */
+  float* lse_planes;  /* device, [n_groups][B,H,S] */
   int32_t t_c[AS_MAX_P * AS_MAX_P];
+  int g, n_groups;
+  uint64_t member[AS_MAX_P * AS_MAX_P];
 } as_cache;
 
-/* Bytes of device memory a cache for these sizes needs (fp32 states only:
- * cache_dt must be AS_F32).  Returns 0 for invalid sizes. */
+/* Bytes of device memory a cache with one entry per pair (g = 1) needs.
+ * cache_dt: AS_F32 or AS_BF16 (the type of the OUT entries).  Returns 0 for
+ * invalid sizes. */
 size_t as_cache_bytes(int B, int H, int S, int d, int P, as_dtype cache_dt);
 
-/* Carve a cache out of `buf` (device, >= as_cache_bytes, 256-byte aligned)
- * and mark every entry empty.  No device access happens here. */
+/* Carve a g = 1 cache out of `buf` (device, >= as_cache_bytes, 256-byte
+ * aligned) and mark every entry empty.  No device access happens here. */
 as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P,
                         as_dtype cache_dt);
 
+/* As as_cache_bytes for groups of g partitions (1 <= g <= P):
+ * n_groups * B*H*S * (d * sizeof(OUT entry) + 4).  Returns 0 for invalid
+ * sizes. */
+size_t as_cache_group_bytes(int B, int H, int S, int d, int P, int g, as_dtype cache_dt);
+
+/* As as_cache_init for groups of g partitions.  AS_ERR_INVALID_ARG for g
+ * outside [1, P] or a short buffer. */
+as_status as_cache_group_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, int g,
+                              as_dtype cache_dt);
+
 /* Check a plan against the cache and derive the reuse bookkeeping, on the host
  * only (no launch, no state change).  h_plan [P*P] row-major (row = query
- * partition).  h_hit[i*P+j] = 1 for reused pairs, else 0; h_age[i*P+j] =
- * step - t_c for reused pairs, else 0.  AS_ERR_CACHE_MISS if a reused entry
- * was never stored; AS_ERR_INVALID_ARG for a code other than 0/1/2. */
+ * partition), one code per pair.  Per (i, G) the code-0 members are the
+ * reused set and the code-2 members the stored set; a group is stored or
+ * reused as a whole.  h_hit[i*P+j] = 1 for reused pairs, else 0;
+ * h_age[i*P+j] = step - t_c(i, j/g) for reused pairs, else 0.  Checks, in
+ * this order: AS_ERR_INVALID_ARG for a code other than 0/1/2, then for a
+ * group with both reused and stored members; AS_ERR_CACHE_MISS if a reused
+ * group was never stored or its reused set differs from the stored member
+ * set. */
 as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step,
                           uint8_t* h_hit, int32_t* h_age);
 
 /* One denoising step's attention under a compute/reuse plan (DiTango review:
  * Core claim; Referee Report, Summary).
- *   final(i) = compose({AS_step(i,j) : plan fresh} U {C(i,j) : plan reuse})
- * written to out [B,H,S,d], lse [B,H,S]; then for AS_PLAN_FRESH_STORE pairs
- * C(i,j) <- AS_step(i,j) (device, in stream order) and t_c(i,j) <- step (host,
- * at return).  h_hit / h_age (may be NULL) as in as_plan_resolve.  The plan is
+ *   C(i,G) <- compose({AS_step(i,j) : j in G, plan AS_PLAN_FRESH_STORE})
+ *             for every group with stored members (OUT rounded to the
+ *             cache type), member(i,G) <- those j, t_c(i,G) <- step;
+ *   final(i) = compose({AS_step(i,j) : plan AS_PLAN_FRESH}
+ *                      U {C(i,G) : G stored or reused by row i})
+ * written to out [B,H,S,d], lse [B,H,S].  Entries are written on the device in
+ * stream order; t_c and member change on the host at return.  With g = 1 and
+ * fp32 entries this is compose over every pair's fresh state or cached
+ * entry.  h_hit / h_age (may be NULL) as in as_plan_resolve.  The plan is
  * checked before any launch: on AS_ERR_CACHE_MISS or AS_ERR_INVALID_ARG
  * nothing is launched and the cache is unchanged.  The cache must have been
  * initialised for the same B, H, S, d, P. */
@@ -237,7 +271,9 @@ as_status as_planner_next(as_planner* pl, const float* local_now, float* local_a
 
 /* After an anchor step (the as_step that used the anchor plan h_plan):
  * measure w and alpha for every pair the plan stored, from the cache, the
- * step's composed LSE lse_full [B,H,S] and local_anchor.  Synchronises. */
+ * step's composed LSE lse_full [B,H,S] and local_anchor.  Synchronises.
+ * The cache must hold one fp32 entry per pair (g = 1, AS_F32), else
+ * AS_ERR_UNSUPPORTED. */
 as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const float* lse_full,
                                    const float* local_anchor, const uint8_t* h_plan, void* scratch,
                                    size_t scratch_bytes, void* stream);

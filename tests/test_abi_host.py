@@ -94,11 +94,65 @@ def test_cache_init_validation(api):
     need = api.as_cache_bytes(1, 2, 64, 64, 4)
     assert L.as_cache_init(ctypes.byref(s), 1 << 20, need - 1, 1, 2, 64, 64, 4, 0) == _lib.AS_ERR_INVALID_ARG
     assert L.as_cache_init(ctypes.byref(s), (1 << 20) + 16, need, 1, 2, 64, 64, 4, 0) == _lib.AS_ERR_INVALID_ARG
-    assert L.as_cache_init(ctypes.byref(s), 1 << 20, need, 1, 2, 64, 64, 4, 1) == _lib.AS_ERR_UNSUPPORTED
+    assert L.as_cache_init(ctypes.byref(s), 1 << 20, need, 1, 2, 64, 64, 4, 7) == _lib.AS_ERR_INVALID_ARG
     assert L.as_cache_init(ctypes.byref(s), 1 << 20, need, 1, 2, 64, 64, 4, 0) == _lib.AS_OK
     assert s.out_planes == 1 << 20
     assert s.lse_planes == (1 << 20) + 4 * 1 * 2 * 64 * 64 * 4
-    assert all(s.t_c[x] == -1 for x in range(16))
+    assert all(s.t_c[x] == -1 for x in range(16)) and s.g == 1 and s.n_groups == 4
+    # bf16 entries: OUT planes of 2-byte elements, LSE planes fp32
+    need_bf = L.as_cache_bytes(1, 2, 64, 64, 4, 1)
+    assert need_bf == 4 * 1 * 2 * 64 * (64 * 2 + 4)
+    assert L.as_cache_init(ctypes.byref(s), 1 << 20, need_bf, 1, 2, 64, 64, 4, 1) == _lib.AS_OK
+    assert s.lse_planes == (1 << 20) + 4 * 1 * 2 * 64 * 64 * 2
+
+
+def test_cache_group_sizes(api):
+    """Grouped caches: ceil(P / g) planes; g outside [1, P] is rejected."""
+    from attention_state_reuse_partition_b200 import _lib
+    L = _lib.LIB
+    rows = 2 * 3 * 120
+    for P, g, dt, esz in [(6, 1, 0, 4), (6, 2, 0, 4), (6, 4, 0, 4), (6, 6, 1, 2), (5, 2, 1, 2)]:
+        NG = (P + g - 1) // g
+        need = L.as_cache_group_bytes(2, 3, 120, 128, P, g, dt)
+        assert need == NG * rows * (128 * esz + 4), (P, g, dt)
+        s = _lib.AsCacheStruct()
+        assert L.as_cache_group_init(ctypes.byref(s), 1 << 24, need, 2, 3, 120, 128, P, g, dt) == _lib.AS_OK
+        assert s.g == g and s.n_groups == NG
+        assert s.lse_planes == (1 << 24) + NG * rows * 128 * esz
+    for g in (0, 7):
+        s = _lib.AsCacheStruct()
+        assert L.as_cache_group_bytes(2, 3, 96, 128, 6, g, 0) == 0
+        assert L.as_cache_group_init(ctypes.byref(s), 1 << 24, 1 << 30, 2, 3, 96, 128, 6, g, 0) == \
+            _lib.AS_ERR_INVALID_ARG
+
+
+def _replay_fixture(api, cache, cases, P, g):
+    """as_plan_resolve against a hand-computed fixture.  Between steps the
+    bookkeeping follows the fixture's rule: every group with stored (code 2)
+    members gets t_c = step and member = those members; a miss or an invalid
+    plan changes nothing."""
+    from attention_state_reuse_partition_b200 import _lib
+    NG = (P + g - 1) // g
+    t_c = np.full((P, NG), -1)
+    member = np.zeros((P, NG), dtype=np.uint64)
+    for c in cases:
+        if c["expect"] in ("cache_miss", "invalid"):
+            with pytest.raises(api.AsError) as ei:
+                api.as_plan_resolve(cache, c["plan"], c["step"])
+            want = _lib.AS_ERR_CACHE_MISS if c["expect"] == "cache_miss" else _lib.AS_ERR_INVALID_ARG
+            assert ei.value.status == want, (c["step"], c["expect"])
+            continue
+        hit, age = api.as_plan_resolve(cache, c["plan"], c["step"])
+        assert np.array_equal(hit, c["hit"]), c["step"]
+        assert np.array_equal(age, c["age"]), c["step"]
+        for i in range(P):
+            for G in range(NG):
+                m = sum(1 << j for j in range(G * g, min((G + 1) * g, P)) if c["plan"][i, j] == 2)
+                if m:
+                    t_c[i, G] = c["step"]
+                    member[i, G] = m
+        cache.set_t_c(t_c)
+        cache.set_member(member)
 
 
 def test_plan_resolve_matches_fixture(api):
@@ -108,23 +162,59 @@ def test_plan_resolve_matches_fixture(api):
     from attention_state_reuse_partition_b200 import _lib
     P, cases = load_plan_fixture()
     cache = api.AsCache.host_only(1, 1, 4 * P, 64, P)
-    t_c = np.full((P, P), -1)
-    for c in cases:
-        if c["expect"] == "cache_miss":
-            with pytest.raises(api.AsError) as ei:
-                api.as_plan_resolve(cache, c["plan"], c["step"])
-            assert ei.value.status == _lib.AS_ERR_CACHE_MISS
-            continue
-        if c["expect"] == "invalid":
-            with pytest.raises(api.AsError) as ei:
-                api.as_plan_resolve(cache, c["plan"], c["step"])
-            assert ei.value.status == _lib.AS_ERR_INVALID_ARG
-            continue
-        hit, age = api.as_plan_resolve(cache, c["plan"], c["step"])
-        assert np.array_equal(hit, c["hit"]), c["step"]
-        assert np.array_equal(age, c["age"]), c["step"]
-        t_c[c["plan"] == 2] = c["step"]
-        cache.set_t_c(t_c)
+    _replay_fixture(api, cache, cases, P, 1)
+
+
+def test_plan_resolve_matches_grouped_fixture(api):
+    """The same for grouped entries (g = 2): member sets, mixed groups."""
+    P, g, cases = load_plan_fixture("plan_grouped_4x4.txt", with_group=True)
+    cache = api.AsCache.host_only(1, 1, 4 * P, 64, P, g=g, cache_dtype="bf16")
+    _replay_fixture(api, cache, cases, P, g)
+
+
+def test_plan_resolve_matches_oracle_on_random_plans(api):
+    """Random plans and group sizes: the C resolve and the oracle agree on
+    hit, age and the kind of error, with the bookkeeping replayed from the
+    oracle's cache."""
+    from oracle import as_oracle as O
+    from attention_state_reuse_partition_b200 import _lib
+    r = np.random.default_rng(11)
+    for trial in range(30):
+        P = int(r.integers(2, 9))
+        g = int(r.integers(1, P + 1))
+        ocache = O.StateCache(P, g)
+        cache = api.AsCache.host_only(1, 1, 2 * P, 64, P, g=g)
+        q = r.normal(size=(1, 1, 2 * P, 2))
+        for t in range(5):
+            plan = r.choice([0, 1, 2], size=(P, P), p=[0.4, 0.3, 0.3]).astype(np.uint8)
+            try:
+                _, _, ohit, oage = O.step(ocache, q, q, q, plan, t, 0.5)
+                oerr = None
+            except O.CacheMiss:
+                oerr = _lib.AS_ERR_CACHE_MISS
+            except O.PlanError:
+                oerr = _lib.AS_ERR_INVALID_ARG
+            try:
+                hit, age = api.as_plan_resolve(cache, plan, t)
+                err = None
+            except api.AsError as e:
+                err = e.status
+            assert err == oerr, (trial, t)
+            if err is None:
+                assert np.array_equal(hit, ohit) and np.array_equal(age, oage), (trial, t)
+            cache.set_t_c(ocache.t_c)
+            cache.set_member([[sum(1 << j for j in m) for m in row] for row in ocache.member])
+
+
+def test_planner_needs_a_pairwise_fp32_cache(api):
+    from attention_state_reuse_partition_b200 import _lib
+    pl = api.AsPlanner(4, 1, 0.5, 0.1)
+    plan = np.ones((4, 4), np.uint8)
+    for g, dt in [(2, "f32"), (1, "bf16")]:
+        cache = api.AsCache.host_only(1, 1, 64, 64, 4, g=g, cache_dtype=dt)
+        st = _lib.LIB.as_planner_commit_anchor(ctypes.byref(pl.struct), ctypes.byref(cache.struct), 1 << 20,
+                                               1 << 20, plan.ctypes.data, 1 << 20, 1 << 30, None)
+        assert st == _lib.AS_ERR_UNSUPPORTED, (g, dt)
 
 
 def test_step_cache_miss_is_reported_before_any_launch(api):

@@ -1,0 +1,151 @@
+"""Grouped cache entries and bf16 entries on the GPU against the float64
+oracle (DiTango review: "If this is right" -- composed states merged into
+coarser groups under memory pressure; ledger: group size g).
+
+Same tolerances as the other parity tests (bf16 inputs: OUT max-abs 2e-2 and
+relative Frobenius 5e-3, LSE max-abs 1e-3; fp32 inputs with fp32 entries:
+1e-5); hit, age, store timestamps and member sets bit-exact.  The oracle rounds its stored entries to bf16 the
+way the kernels do (round to nearest even), so both sides compose the same
+cached values up to accumulation order."""
+import numpy as np
+import pytest
+import torch
+
+from attention_state_reuse_partition_b200 import workloads as W
+from oracle import as_oracle as O
+from tests.test_gpu_parity import check_bf16, check_f32, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    from attention_state_reuse_partition_b200 import build
+    build.build()
+    from attention_state_reuse_partition_b200 import api as a
+    return a
+
+
+def _members(ocache):
+    return np.array([[sum(1 << j for j in m) for m in row] for row in ocache.member], dtype=np.uint64)
+
+
+def _run_grouped(api, s, qkv_steps, plans, g, cache_dt, rows=None, heads=None, dtype_check=check_bf16):
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=g, cache_dtype=cache_dt)
+    ocache = O.StateCache(s.P, g, "bf16" if cache_dt == "bf16" else "f32")
+    for t, (q, k, v) in enumerate(qkv_steps):
+        plan = np.asarray(plans[t])
+        out, lse, hit, age = api.as_step(cache, q, k, v, plan, t)
+        torch.cuda.synchronize()
+        hs = slice(None) if heads is None else heads
+        qn = f64(q[:, hs])
+        kn, vn = f64(k[:, hs]), f64(v[:, hs])
+        r = np.arange(s.S) if rows is None else np.asarray(rows)
+        ref_o, ref_l, ref_hit, ref_age = O.step(ocache, qn, kn, vn, plan, t, s.scale, rows=r)
+        assert np.array_equal(hit, ref_hit), f"hit at step {t}"
+        assert np.array_equal(age, ref_age), f"age at step {t}"
+        assert np.array_equal(cache.t_c, ocache.t_c), f"t_c at step {t}"
+        assert np.array_equal(cache.member, _members(ocache)), f"members at step {t}"
+        rt = torch.as_tensor(r, device=out.device)
+        dtype_check(out[:, hs][:, :, rt], lse[:, hs][:, :, rt], ref_o, ref_l, f"g={g} {cache_dt} step {t}")
+    return cache
+
+
+@pytest.mark.parametrize("g", [2, 3, 4, 16])
+@pytest.mark.parametrize("cache_dt", ["f32", "bf16"])
+def test_step_grouped_video_long_small(api, g, cache_dt):
+    """Four steps of the long-trajectory construction (forced pairs lift whole
+    groups to fresh-and-store); g = 3 leaves a short last group, g = 16 puts
+    every partition in one group."""
+    s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16)
+    steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
+    plans = [W.grouped_plan_for_step(s, t, g).numpy() for t in range(s.steps)]
+    assert any((p == W.PLAN_REUSE).any() for p in plans[1:])
+    _run_grouped(api, s, steps, plans, g, cache_dt)
+
+
+@pytest.mark.parametrize("g", [1, 4])
+def test_step_bf16_cache_video_reuse_small(api, g):
+    s = W.spec("video_reuse", H=2, rows=12, cols=16, S=16 * 12 * 16)
+    steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
+    plans = [W.grouped_plan_for_step(s, t, g).numpy() for t in range(s.steps)]
+    _run_grouped(api, s, steps, plans, g, "bf16")
+
+
+def test_step_grouped_f32_inputs(api):
+    """fp32 inputs (CUDA-core path) with grouped fp32 entries: 1e-5."""
+    s = W.spec("tiny_f32", P=8)
+    q, k, v = (x.cuda() for x in W.iid_qkv(s))
+    k2 = k + 0.1 * torch.randn(k.shape, generator=torch.Generator(device="cuda").manual_seed(5), device="cuda")
+    near = np.abs(np.arange(8)[:, None] - np.arange(8)[None, :]) <= 1
+    plans = [np.where(near, 1, 2).astype(np.uint8), np.where(near, 1, 0).astype(np.uint8)]
+    _run_grouped(api, s, [(q, k, v), (q, k2, v)], plans, 3, "f32", dtype_check=check_f32)
+
+
+def test_step_grouped_fixture_on_gpu(api):
+    """The hand-computed grouped fixture through as_step with bf16 entries:
+    bit-exact bookkeeping, errors leave the cache unchanged, and every step's
+    states match the oracle."""
+    from tests._golden import load_plan_fixture
+    from attention_state_reuse_partition_b200 import _lib
+    P, g, cases = load_plan_fixture("plan_grouped_4x4.txt", with_group=True)
+    s = W.spec("flux_image", H=2, S=64 * P, d=64, P=P)
+    q, k, v = (x.cuda() for x in W.flux_qkv(s))
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=g, cache_dtype="bf16")
+    ocache = O.StateCache(P, g, "bf16")
+    qn, kn, vn = (f64(x) for x in (q, k, v))
+    for c in cases:
+        if c["expect"] in ("cache_miss", "invalid"):
+            before = (cache.t_c, cache.member)
+            with pytest.raises(api.AsError) as ei:
+                api.as_step(cache, q, k, v, c["plan"], c["step"])
+            want = _lib.AS_ERR_CACHE_MISS if c["expect"] == "cache_miss" else _lib.AS_ERR_INVALID_ARG
+            assert ei.value.status == want
+            assert np.array_equal(cache.t_c, before[0]) and np.array_equal(cache.member, before[1])
+            continue
+        out, lse, hit, age = api.as_step(cache, q, k, v, c["plan"], c["step"])
+        assert np.array_equal(hit, c["hit"]) and np.array_equal(age, c["age"])
+        ref_o, ref_l, _, _ = O.step(ocache, qn, kn, vn, c["plan"], c["step"], s.scale)
+        check_bf16(out, lse, ref_o, ref_l, f"grouped fixture step {c['step']}")
+        assert np.array_equal(cache.t_c, ocache.t_c) and np.array_equal(cache.member, _members(ocache))
+
+
+def test_bf16_entries_are_the_rounded_fp32_entries(api):
+    """The same anchor step with an fp32 and a bf16 cache: every bf16 entry is
+    the round-to-nearest-even bf16 of the fp32 entry (bit-exact: both come
+    from the same kernel arithmetic), and the LSE planes are identical."""
+    s = W.spec("video_reuse", H=2, rows=4, cols=8, S=16 * 4 * 8)
+    _, q, k, v = next(iter(W.video_trajectory(s)))
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    plan = W.grouped_plan_for_step(s, 0, 4).numpy()
+    c32 = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=4, cache_dtype="f32")
+    c16 = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=4, cache_dtype="bf16")
+    api.as_step(c32, q, k, v, plan, 0)
+    api.as_step(c16, q, k, v, plan, 0)
+    torch.cuda.synchronize()
+    o32, l32 = c32.planes()
+    o16, l16 = c16.planes()
+    stored = torch.zeros(((s.P + 3) // 4, s.S), dtype=torch.bool)  # [group plane, token]
+    for i in range(s.P):
+        for G in range(stored.shape[0]):
+            if (plan[i, G * 4:(G + 1) * 4] == W.PLAN_FRESH_STORE).any():
+                stored[G, i * s.n:(i + 1) * s.n] = True
+    stored = stored.cuda()
+    a = o32.permute(0, 3, 1, 2, 4)[stored]
+    b = o16.permute(0, 3, 1, 2, 4)[stored]
+    assert a.numel() > 0
+    assert torch.equal(a.to(torch.bfloat16), b)
+    assert torch.equal(l32.permute(0, 3, 1, 2)[stored], l16.permute(0, 3, 1, 2)[stored])
+
+
+def test_step_grouped_video_long_full(api):
+    """video_long at full size with g = 4 and bf16 entries (a 5.4 GB cache
+    instead of 43.3 GB): seeded samples of 4 rows per partition on two heads
+    against the oracle, and the whole bookkeeping bit-exact."""
+    s = W.spec("video_long")
+    steps = [(q, k, v) for _, q, k, v in W.video_trajectory(s, device="cuda")]
+    plans = [W.grouped_plan_for_step(s, t, 4).numpy() for t in range(s.steps)]
+    cache = _run_grouped(api, s, steps, plans, 4, "bf16", rows=W.sample_rows(s, 4).numpy(), heads=[0, 39])
+    assert cache.buffer.numel() == api.as_cache_bytes(s.B, s.H, s.S, s.d, s.P, 4, "bf16")
+    del steps, cache
+    torch.cuda.empty_cache()
