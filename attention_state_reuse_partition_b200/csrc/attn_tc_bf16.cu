@@ -50,6 +50,7 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
 #define ASP_POLY_PAIR_EVERY 0
 #endif
 constexpr int POLY_PAIR_EVERY = ASP_POLY_PAIR_EVERY;  // every n-th pair of exponentials on the FMA pipe
+constexpr int POLY_PERIOD = POLY_PAIR_EVERY > 0 ? POLY_PAIR_EVERY : 1;
 // registers: launched at LAUNCH_REGS per thread; the control warpgroup (TMA,
 // MMA, two idle warps) gives up registers to the softmax warpgroups.
 // 128 * CTRL_REGS + 128 * NQ * SOFTMAX_REGS == NTHREADS * LAUNCH_REGS
@@ -400,7 +401,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float x0, x1;
         f2_unpack(x2, x0, x1);
         uint64_t p2;
-        if (POLY_PAIR_EVERY > 0 && i % POLY_PAIR_EVERY == POLY_PAIR_EVERY - 1)
+        if (POLY_PAIR_EVERY > 0 && i % POLY_PERIOD == POLY_PERIOD - 1)
           p2 = exp2_poly2(x0, x1);
         else
           p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
