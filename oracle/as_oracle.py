@@ -336,6 +336,10 @@ def mse(a, b):
 #   floor(R * count) with the smallest ASE are reused (threshold = that
 #   order statistic), ties broken by (i, j); the others are fresh and refresh
 #   their cache entry;
+# * with cache groups (Eq. 12, ASE of a group G_i) the unit is a group's set
+#   of remote members: w and alpha come from its composed entry (w of the
+#   group is the sum of its members' weights), and the selection above runs
+#   over these units;
 # * an anchor is taken when no anchor exists or when the relative local drift
 #   max_i D(i,t) / ||OUT_ta(i,i)||_F exceeds eps_local; at an anchor every pair
 #   is fresh and every remote pair is stored.
@@ -370,22 +374,31 @@ def ase(w, alpha, drift):
         np.asarray(drift, dtype=np.float64)[:, None]
 
 
-def select_plan(ase_ij, window, reuse_ratio):
-    """Plan codes from ASE values (see the readings above)."""
+def select_plan(ase_ij, window, reuse_ratio, g=1):
+    """Plan codes from ASE values (see the readings above).
+
+    With cache groups of g partitions the planner decides per group (Eq. 12:
+    ASE of a group G_i): ase_ij is [P, n_groups(P, g)], the units are the
+    groups (i, G) with at least one member outside the window, and a unit's
+    remote members are reused or stored together; members inside the window
+    stay fresh.  g = 1 is the per-pair selection."""
     ase_ij = np.asarray(ase_ij, dtype=np.float64)
     P = ase_ij.shape[0]
     plan = np.full((P, P), PLAN_FRESH_STORE, dtype=np.uint8)
-    remote = []
+    units = []
     for i in range(P):
         for j in range(P):
             if abs(i - j) <= window:
                 plan[i, j] = PLAN_FRESH
-            else:
-                remote.append((ase_ij[i, j], i, j))
-    remote.sort()
-    n_reuse = int(np.floor(reuse_ratio * len(remote) + 1e-9))
-    for _, i, j in remote[:n_reuse]:
-        plan[i, j] = PLAN_REUSE
+        for G in range(n_groups(P, g)):
+            if any(abs(i - j) > window for j in range(G * g, min((G + 1) * g, P))):
+                units.append((ase_ij[i, G], i, G))
+    units.sort()
+    n_reuse = int(np.floor(reuse_ratio * len(units) + 1e-9))
+    for _, i, G in units[:n_reuse]:
+        for j in range(G * g, min((G + 1) * g, P)):
+            if abs(i - j) > window:
+                plan[i, j] = PLAN_REUSE
     return plan
 
 
@@ -400,12 +413,12 @@ class Planner:
     """The planner's state between steps: the anchor's w, alpha and local
     states (OUT_ta(i,i) for every i, [B,H,S,d])."""
 
-    def __init__(self, P, window, reuse_ratio, eps_local):
-        self.P, self.window = P, window
+    def __init__(self, P, window, reuse_ratio, eps_local, g=1):
+        self.P, self.window, self.g = P, window, g
         self.reuse_ratio, self.eps_local = reuse_ratio, eps_local
         self.has_anchor = False
-        self.w = np.zeros((P, P))
-        self.alpha = np.zeros((P, P))
+        self.w = np.zeros((P, n_groups(P, g)))
+        self.alpha = np.zeros((P, n_groups(P, g)))
         self.local_anchor = None
 
 
@@ -427,23 +440,24 @@ def planner_next(pl, local_now, n):
         pl.local_anchor = np.array(local_now, dtype=np.float64, copy=True)
         return anchor_plan(P, pl.window), True, drift, None
     a = ase(pl.w, pl.alpha, drift)
-    return select_plan(a, pl.window, pl.reuse_ratio), False, drift, a
+    return select_plan(a, pl.window, pl.reuse_ratio, pl.g), False, drift, a
 
 
 def planner_commit_anchor(pl, cache, lse_full, rows_of, n):
-    """After an anchor step: w and alpha of every stored pair from the cache
-    entries, the composed LSE and the anchor's local states.  ``rows_of(i)``
-    gives the positions, within the evaluated rows, of partition i's rows
-    (the same rows the cache entries hold)."""
+    """After an anchor step: w and alpha of every stored entry (a pair, or a
+    group of remote members: its composed state stands for the group, Eq. 12)
+    from the cache entries, the composed LSE and the anchor's local states.
+    ``rows_of(i)`` gives the positions, within the evaluated rows, of
+    partition i's rows (the same rows the cache entries hold)."""
     P = pl.P
     for i in range(P):
         sel = rows_of(i)
         local = pl.local_anchor[..., i * n:(i + 1) * n, :]
         local_norm = frob(local)
-        for j in range(P):
-            if (i, j) not in cache.entry or cache.t_c[i, j] < 0 or abs(i - j) <= pl.window:
+        for G in range(n_groups(P, pl.g)):
+            if (i, G) not in cache.entry or cache.t_c[i, G] < 0:
                 continue
-            o, l = cache.entry[(i, j)]
-            pl.w[i, j] = float(np.mean(np.exp(np.asarray(l) - np.asarray(lse_full)[..., sel])))
-            pl.alpha[i, j] = frob(o) / local_norm
+            o, l = cache.entry[(i, G)]
+            pl.w[i, G] = float(np.mean(np.exp(np.asarray(l) - np.asarray(lse_full)[..., sel])))
+            pl.alpha[i, G] = frob(o) / local_norm
     pl.has_anchor = True

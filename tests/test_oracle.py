@@ -457,12 +457,79 @@ def pin_planner_trajectory(o):
     assert anchor2, "a large local drift must trigger an anchor"
 
 
+def pin_planner_group_weights(o):
+    """Grouped anchor statistics: the weight of a group entry is the sum of
+    its members' weights (exp of a composed LSE is the sum of the members'
+    exps), computed here from scipy log-sum-exps of the raw scores; alpha is
+    the Frobenius-norm ratio of the group's composed OUT."""
+    r = _rng(35)
+    B, H, S, d, P, g = 1, 2, 48, 8, 6, 2
+    n = S // P
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    pl = o.Planner(P, window=1, reuse_ratio=0.5, eps_local=0.1, g=g)
+    cache = o.StateCache(P, g)
+    local = np.concatenate([o.attention_state(q[..., i * n:(i + 1) * n, :], k[..., i * n:(i + 1) * n, :],
+                                              v[..., i * n:(i + 1) * n, :], 0.3)[0] for i in range(P)], axis=-2)
+    plan0, anchor0, _, _ = o.planner_next(pl, local, n)
+    assert anchor0
+    _, lse0, _, _ = o.step(cache, q, k, v, plan0, 0, 0.3)
+    o.planner_commit_anchor(pl, cache, lse0, lambda i: np.arange(i * n, (i + 1) * n), n)
+    sc = 0.3 * np.einsum("bhqd,bhkd->bhqk", q, k)
+    full = scipy.special.logsumexp(sc, axis=-1)
+    for i in range(P):
+        rows = slice(i * n, (i + 1) * n)
+        for G in range(P // g):
+            remote = [j for j in range(G * g, (G + 1) * g) if abs(i - j) > 1]
+            if not remote:
+                assert pl.w[i, G] == 0.0
+                continue
+            w_sum = sum(float(np.mean(np.exp(scipy.special.logsumexp(sc[..., rows, j * n:(j + 1) * n], axis=-1)
+                                             - full[..., rows]))) for j in remote)
+            _close(pl.w[i, G], w_sum, 1e-12, f"group weight ({i},{G})")
+
+
+def pin_planner_select_grouped(o):
+    """Selection over groups, worked by hand: P = 4, g = 2, window 0, R = 0.5.
+    Units (8, each with a remote member) sorted by ASE: (2,1) (0,0) (1,0)
+    (2,0) are reused; window members stay fresh, the rest are stored."""
+    a = np.array([[0.1, 0.5], [0.2, 0.9], [0.3, 0.05], [0.8, 0.4]])
+    want = np.array([[1, 0, 2, 2], [0, 1, 2, 2], [0, 0, 1, 0], [2, 2, 2, 1]], np.uint8)
+    assert np.array_equal(o.select_plan(a, 0, 0.5, 2), want), o.select_plan(a, 0, 0.5, 2)
+    assert (o.select_plan(a, 0, 0.0, 2) != o_REUSE).all()
+    # groups fully inside the window are no unit: window 1 leaves (0,1)...(3,0) as units only
+    full = o.select_plan(a, 1, 1.0, 2)
+    assert np.array_equal(full, np.array([[1, 1, 0, 0], [1, 1, 1, 0], [0, 1, 1, 1], [0, 0, 1, 1]], np.uint8))
+
+
+def pin_planner_trajectory_grouped(o):
+    """The trajectory pin with groups of 2: an anchor, then a reuse of
+    floor(R * #units) units of unchanged inputs that equals full attention."""
+    r = _rng(36)
+    B, H, S, d, P, g = 1, 1, 48, 4, 6, 2
+    n = S // P
+    q, k, v = (r.normal(size=(B, H, S, d)) for _ in range(3))
+    pl = o.Planner(P, window=0, reuse_ratio=0.5, eps_local=0.05, g=g)
+    cache = o.StateCache(P, g)
+    local = np.concatenate([o.attention_state(q[..., i * n:(i + 1) * n, :], k[..., i * n:(i + 1) * n, :],
+                                              v[..., i * n:(i + 1) * n, :], 0.5)[0] for i in range(P)], axis=-2)
+    plan0, _, _, _ = o.planner_next(pl, local, n)
+    _, lse0, _, _ = o.step(cache, q, k, v, plan0, 0, 0.5)
+    o.planner_commit_anchor(pl, cache, lse0, lambda i: np.arange(i * n, (i + 1) * n), n)
+    plan1, anchor1, _, _ = o.planner_next(pl, local, n)
+    assert not anchor1
+    reused_units = sum(bool((plan1[i, G * g:(G + 1) * g] == o_REUSE).any()) for i in range(P) for G in range(P // g))
+    assert reused_units == (P * (P // g)) // 2, reused_units   # every (i, G) has a remote member at window 0
+    out1, _, _, _ = o.step(cache, q, k, v, plan1, 1, 0.5)
+    _close(out1, _sdpa(q, k, v, 0.5), TOL, "grouped planner reuse of unchanged states")
+
+
 PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_forms,
         pin_compose_closed, pin_assoc_comm, pin_split_invariance, pin_single_partition,
         pin_plan_golden, pin_step_all_fresh, pin_step_reuse_identical, pin_step_reuse_mixed,
         pin_planner_weights, pin_planner_ratios, pin_planner_drift, pin_planner_select, pin_planner_trajectory,
         pin_round_bf16, pin_plan_grouped_golden, pin_step_grouped_identical, pin_step_grouped_mixed,
-        pin_step_bf16_cache]
+        pin_step_bf16_cache,
+        pin_planner_group_weights, pin_planner_select_grouped, pin_planner_trajectory_grouped]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -569,6 +636,18 @@ def _m_groups_floor(P, g):
     return P // g
 
 
+def _m_select_group_window(ase_ij, window, reuse_ratio, g=1):
+    plan = _orig["select_plan"](ase_ij, window, reuse_ratio, g)
+    P = plan.shape[0]
+    for i in range(P):
+        for G in range((P + g - 1) // g):
+            js = range(G * g, min((G + 1) * g, P))
+            if any(plan[i, j] == 0 for j in js):
+                for j in js:
+                    plan[i, j] = 0
+    return plan
+
+
 def _m_store_all_fresh(cache, q, k, v, plan, t, scale, rows=None):
     res = _orig["step"](cache, q, k, v, plan, t, scale, rows)
     cache.t_c[np.asarray(plan) == 1] = t
@@ -596,12 +675,12 @@ def _m_drift_relative(out_now, out_anchor):
     return (d / nrm if nrm > 0 else 0.0), nrm
 
 
-def _m_select_largest(ase_ij, window, reuse_ratio):
-    return _orig["select_plan"](-np.asarray(ase_ij), window, reuse_ratio)
+def _m_select_largest(ase_ij, window, reuse_ratio, g=1):
+    return _orig["select_plan"](-np.asarray(ase_ij), window, reuse_ratio, g)
 
 
-def _m_select_window(ase_ij, window, reuse_ratio):
-    return _orig["select_plan"](ase_ij, window - 1, reuse_ratio)
+def _m_select_window(ase_ij, window, reuse_ratio, g=1):
+    return _orig["select_plan"](ase_ij, window - 1, reuse_ratio, g)
 
 
 def _m_ase_no_alpha(w, alpha, drift):
@@ -632,6 +711,7 @@ MUTANTS = {
     "round_bf16: truncates": ("round_bf16", _m_bf16_truncate),
     "round_bf16: no rounding": ("round_bf16", _m_bf16_not_rounded),
     "n_groups: drops the short last group": ("n_groups", _m_groups_floor),
+    "select_plan: a reused group takes its window members too": ("select_plan", _m_select_group_window),
 }
 
 
