@@ -24,7 +24,7 @@ EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as
            "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe",
            "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
            "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static",
-           "as_cache_group_bytes", "as_cache_group_init")
+           "as_cache_group_bytes", "as_cache_group_init", "as_planner_group_init", "as_plan_select_grouped")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -50,6 +50,7 @@ class AsPlannerStruct(ctypes.Structure):
         ("alpha", ctypes.c_double * (AS_MAX_P * AS_MAX_P)),
         ("drift", ctypes.c_double * AS_MAX_P),
         ("rel_drift", ctypes.c_double * AS_MAX_P),
+        ("g", ctypes.c_int),
     ]
 
 
@@ -96,6 +97,10 @@ def _load() -> ctypes.CDLL:
     dbl = ctypes.c_double
     lib.as_planner_init.restype = c_int
     lib.as_planner_init.argtypes = [ctypes.POINTER(AsPlannerStruct), c_int, c_int, dbl, dbl]
+    lib.as_planner_group_init.restype = c_int
+    lib.as_planner_group_init.argtypes = [ctypes.POINTER(AsPlannerStruct), c_int, c_int, c_int, dbl, dbl]
+    lib.as_plan_select_grouped.restype = c_int
+    lib.as_plan_select_grouped.argtypes = [vp, c_int, c_int, c_int, dbl, vp]
     lib.as_planner_scratch_bytes.restype = sz
     lib.as_planner_scratch_bytes.argtypes = [c_int, c_int, c_int]
     lib.as_local_states.restype = c_int

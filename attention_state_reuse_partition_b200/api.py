@@ -214,10 +214,12 @@ class AsPlanner:
     local states), allocated with torch."""
 
     def __init__(self, P: int, window: int, reuse_ratio: float, eps_local: float, B: int = 0, H: int = 0,
-                 S: int = 0, d: int = 0, device="cuda"):
+                 S: int = 0, d: int = 0, device="cuda", g: int = 1):
         self.struct = AsPlannerStruct()
-        check(LIB.as_planner_init(ctypes.byref(self.struct), P, window, float(reuse_ratio), float(eps_local)))
-        self.P = P
+        check(LIB.as_planner_group_init(ctypes.byref(self.struct), P, g, window, float(reuse_ratio),
+                                        float(eps_local)))
+        self.P, self.g = P, g
+        self.NG = (P + g - 1) // g
         self.scratch = None
         self.local_anchor = None
         if B:
@@ -234,11 +236,13 @@ class AsPlanner:
 
     @property
     def w(self):
-        return self._arr("w", self.P * self.P).reshape(self.P, self.P)
+        """w(i, G) of the last anchor, [P, n_groups]."""
+        return self._arr("w", self.P * self.NG).reshape(self.P, self.NG)
 
     @property
     def alpha(self):
-        return self._arr("alpha", self.P * self.P).reshape(self.P, self.P)
+        """alpha(i, G) of the last anchor, [P, n_groups]."""
+        return self._arr("alpha", self.P * self.NG).reshape(self.P, self.NG)
 
     @property
     def drift(self):
@@ -249,8 +253,8 @@ class AsPlanner:
         return self._arr("rel_drift", self.P)
 
 
-def as_planner_init(P, window, reuse_ratio, eps_local, B=0, H=0, S=0, d=0, device="cuda") -> AsPlanner:
-    return AsPlanner(P, window, reuse_ratio, eps_local, B, H, S, d, device)
+def as_planner_init(P, window, reuse_ratio, eps_local, B=0, H=0, S=0, d=0, device="cuda", g=1) -> AsPlanner:
+    return AsPlanner(P, window, reuse_ratio, eps_local, B, H, S, d, device, g)
 
 
 def as_local_states(q, k, v, P: int, scale: Optional[float] = None, out=None, lse=None, stream=None):
@@ -289,26 +293,29 @@ def as_plan_drift_static(now, anchor, P: int, stream=None):
     return drift, norm
 
 
-def as_plan_select(ase, window: int, reuse_ratio: float):
-    """Host-only plan selection from ASE values [P, P]."""
+def as_plan_select(ase, window: int, reuse_ratio: float, g: int = 1):
+    """Host-only plan selection from ASE values [P, n_groups] (groups of g
+    KV partitions; [P, P] for g = 1); returns the plan [P, P]."""
     a = np.ascontiguousarray(np.asarray(ase, dtype=np.float64))
     P = a.shape[0]
+    if a.shape != (P, (P + g - 1) // g):
+        raise AsError(_lib.AS_ERR_INVALID_ARG, f"ASE must be [P, ceil(P/g)], got {a.shape}")
     plan = np.zeros(P * P, dtype=np.uint8)
-    check(LIB.as_plan_select(a.ctypes.data, P, int(window), float(reuse_ratio), plan.ctypes.data))
+    check(LIB.as_plan_select_grouped(a.ctypes.data, P, int(g), int(window), float(reuse_ratio), plan.ctypes.data))
     return plan.reshape(P, P)
 
 
 def as_planner_next(pl: AsPlanner, local_now, stream=None):
-    """(plan [P,P], is_anchor, ase [P,P]) of the next step."""
+    """(plan [P,P], is_anchor, ase [P, n_groups]) of the next step."""
     B, H, S, d = local_now.shape
     P = pl.P
     plan = np.zeros(P * P, dtype=np.uint8)
-    ase = np.zeros(P * P, dtype=np.float64)
+    ase = np.zeros(P * pl.NG, dtype=np.float64)
     is_anchor = ctypes.c_int(0)
     check(LIB.as_planner_next(ctypes.byref(pl.struct), _dev(local_now, "local_now"), _dev(pl.local_anchor, "anchor"),
                               B, H, S, d, _dev(pl.scratch, "scratch"), pl.scratch.numel() * 8, plan.ctypes.data,
                               ctypes.byref(is_anchor), ase.ctypes.data, _stream_ptr(stream)))
-    return plan.reshape(P, P), bool(is_anchor.value), ase.reshape(P, P)
+    return plan.reshape(P, P), bool(is_anchor.value), ase.reshape(P, pl.NG)
 
 
 def as_planner_commit_anchor(pl: AsPlanner, cache: AsCache, lse_full, plan, stream=None):

@@ -139,23 +139,29 @@ as_status check_scratch(void* scratch, size_t bytes, int B, int H, int P) {
   return AS_OK;
 }
 
-// selection from ASE values: |i-j| <= window fresh; of the rest the
-// floor(R * count) smallest (ties by (i, j)) reused, the others fresh + stored
-void select_plan(const double* ase, int P, int window, double ratio, uint8_t* plan) {
-  std::vector<std::tuple<double, int, int>> remote;
-  for (int i = 0; i < P; ++i)
-    for (int j = 0; j < P; ++j) {
-      if (std::abs(i - j) <= window) {
-        plan[i * P + j] = AS_PLAN_FRESH;
-      } else {
-        plan[i * P + j] = AS_PLAN_FRESH_STORE;
-        remote.emplace_back(ase[i * P + j], i, j);
-      }
+// selection from ASE values per (i, G) unit (groups of g KV partitions, ase
+// [P][NG]): |i-j| <= window fresh; the units are the groups with a member
+// outside the window; the floor(R * count) units with the smallest ASE (ties
+// by (i, G)) have their remote members reused, the others stored
+void select_plan(const double* ase, int P, int g, int window, double ratio, uint8_t* plan) {
+  const int NG = (P + g - 1) / g;
+  std::vector<std::tuple<double, int, int>> units;
+  for (int i = 0; i < P; ++i) {
+    for (int j = 0; j < P; ++j)
+      plan[i * P + j] = std::abs(i - j) <= window ? AS_PLAN_FRESH : AS_PLAN_FRESH_STORE;
+    for (int G = 0; G < NG; ++G) {
+      bool remote = false;
+      for (int j = G * g; j < std::min((G + 1) * g, P); ++j) remote |= std::abs(i - j) > window;
+      if (remote) units.emplace_back(ase[i * NG + G], i, G);
     }
-  std::sort(remote.begin(), remote.end());
-  const size_t n_reuse = static_cast<size_t>(std::floor(ratio * static_cast<double>(remote.size()) + 1e-9));
-  for (size_t x = 0; x < n_reuse && x < remote.size(); ++x)
-    plan[std::get<1>(remote[x]) * P + std::get<2>(remote[x])] = AS_PLAN_REUSE;
+  }
+  std::sort(units.begin(), units.end());
+  const size_t n_reuse = static_cast<size_t>(std::floor(ratio * static_cast<double>(units.size()) + 1e-9));
+  for (size_t x = 0; x < n_reuse && x < units.size(); ++x) {
+    const int i = std::get<1>(units[x]), G = std::get<2>(units[x]);
+    for (int j = G * g; j < std::min((G + 1) * g, P); ++j)
+      if (std::abs(i - j) > window) plan[i * P + j] = AS_PLAN_REUSE;
+  }
 }
 
 void anchor_plan(int P, int window, uint8_t* plan) {
@@ -440,9 +446,10 @@ as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream) {
   return ok();
 }
 
-as_status as_planner_init(as_planner* pl, int P, int window, double reuse_ratio, double eps_local) {
+as_status as_planner_group_init(as_planner* pl, int P, int g, int window, double reuse_ratio, double eps_local) {
   if (!pl) return fail(AS_ERR_INVALID_ARG, "null planner");
   if (P < 1 || P > AS_MAX_P) return fail(AS_ERR_INVALID_ARG, "P must be in [1, %d]", AS_MAX_P);
+  if (g < 1 || g > P) return fail(AS_ERR_INVALID_ARG, "group size %d outside [1, %d]", g, P);
   if (window < 0) return fail(AS_ERR_INVALID_ARG, "window must be >= 0");
   if (!(reuse_ratio >= 0.0 && reuse_ratio <= 1.0)) return fail(AS_ERR_INVALID_ARG, "reuse_ratio must be in [0, 1]");
   if (!(eps_local >= 0.0)) return fail(AS_ERR_INVALID_ARG, "eps_local must be >= 0");
@@ -452,7 +459,12 @@ as_status as_planner_init(as_planner* pl, int P, int window, double reuse_ratio,
   pl->window = window;
   pl->reuse_ratio = reuse_ratio;
   pl->eps_local = eps_local;
+  pl->g = g;
   return ok();
+}
+
+as_status as_planner_init(as_planner* pl, int P, int window, double reuse_ratio, double eps_local) {
+  return as_planner_group_init(pl, P, 1, window, reuse_ratio, eps_local);
 }
 
 size_t as_planner_scratch_bytes(int B, int H, int P) {
@@ -540,12 +552,17 @@ as_status as_plan_drift_static(const float* now, const float* anchor, int B, int
   return ok();
 }
 
-as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan) {
+as_status as_plan_select_grouped(const double* h_ase, int P, int g, int window, double reuse_ratio,
+                                 uint8_t* h_plan) {
   if (!h_ase || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
-  if (P < 1 || P > AS_MAX_P || window < 0 || !(reuse_ratio >= 0.0 && reuse_ratio <= 1.0))
-    return fail(AS_ERR_INVALID_ARG, "bad P, window or reuse_ratio");
-  select_plan(h_ase, P, window, reuse_ratio, h_plan);
+  if (P < 1 || P > AS_MAX_P || g < 1 || g > P || window < 0 || !(reuse_ratio >= 0.0 && reuse_ratio <= 1.0))
+    return fail(AS_ERR_INVALID_ARG, "bad P, g, window or reuse_ratio");
+  select_plan(h_ase, P, g, window, reuse_ratio, h_plan);
   return ok();
+}
+
+as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan) {
+  return as_plan_select_grouped(h_ase, P, 1, window, reuse_ratio, h_plan);
 }
 
 as_status as_planner_next(as_planner* pl, const float* local_now, float* local_anchor, int B, int H, int S, int d,
@@ -573,17 +590,18 @@ as_status as_planner_next(as_planner* pl, const float* local_now, float* local_a
     }
     anchor = worst > pl->eps_local;
   }
-  if (h_ase) std::memset(h_ase, 0, static_cast<size_t>(P) * P * sizeof(double));
+  const int g = pl->g, NG = (P + g - 1) / g;
+  if (h_ase) std::memset(h_ase, 0, static_cast<size_t>(P) * NG * sizeof(double));
   if (anchor) {
     anchor_plan(P, pl->window, h_plan);
     const size_t bytes = static_cast<size_t>(B) * H * S * d * sizeof(float);
     cudaError_t e = cudaMemcpyAsync(local_anchor, local_now, bytes, cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "anchor local-state copy");
   } else {
-    std::vector<double> a(static_cast<size_t>(P) * P);
+    std::vector<double> a(static_cast<size_t>(P) * NG);
     for (int i = 0; i < P; ++i)
-      for (int j = 0; j < P; ++j) a[i * P + j] = pl->w[i * P + j] * pl->alpha[i * P + j] * pl->drift[i];
-    select_plan(a.data(), P, pl->window, pl->reuse_ratio, h_plan);
+      for (int G = 0; G < NG; ++G) a[i * NG + G] = pl->w[i * NG + G] * pl->alpha[i * NG + G] * pl->drift[i];
+    select_plan(a.data(), P, g, pl->window, pl->reuse_ratio, h_plan);
     if (h_ase) std::memcpy(h_ase, a.data(), a.size() * sizeof(double));
   }
   *h_is_anchor = anchor ? 1 : 0;
@@ -598,25 +616,26 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
   if ((s = check_cache(c)) != AS_OK) return s;
   const int P = pl->P;
   if (c->P != P) return fail(AS_ERR_INVALID_ARG, "cache and planner disagree on P");
-  if (c->g != 1 || c->cache_dt != AS_F32)
-    return fail(AS_ERR_UNSUPPORTED, "the anchor statistics read per-pair fp32 entries: the cache needs g = 1 and AS_F32");
+  if (c->g != pl->g)
+    return fail(AS_ERR_INVALID_ARG, "cache groups of %d partitions, planner groups of %d", c->g, pl->g);
   if (!lse_full || !local_anchor || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
   const int B = c->B, H = c->H, S = c->S, d = c->d, n = S / P;
   if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // units: the (i, G) entries this anchor stored
+  const int g = c->g, NG = c->n_groups;
   asp::PlanRows sel;
   std::memset(&sel, 0, sizeof(sel));
   for (int i = 0; i < P; ++i)
-    for (int j = 0; j < P; ++j)
-      sel.v[i * P + j] = (h_plan[i * P + j] == AS_PLAN_FRESH_STORE && std::abs(i - j) > pl->window) ? 1 : 0;
+    for (int G = 0; G < NG; ++G) sel.v[i * NG + G] = group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE) ? 1 : 0;
   double* partials = static_cast<double*>(scratch);
-  double* sums = partials + static_cast<size_t>(P) * P * B * H * 2;
-  cudaError_t e = asp::launch_anchor_stats(static_cast<const float*>(c->out_planes), c->lse_planes, lse_full,
+  double* sums = partials + static_cast<size_t>(P) * NG * B * H * 2;
+  cudaError_t e = asp::launch_anchor_stats(c->out_planes, c->cache_dt == AS_BF16, c->lse_planes, lse_full,
                                            static_cast<long long>(B) * H * S * d, static_cast<long long>(B) * H * S,
-                                           P, B * H, S, d, sel, partials, sums, st);
+                                           P, NG, B * H, S, d, sel, partials, sums, st);
   if (e != cudaSuccess) return cuda_fail(e, "anchor statistics launch");
-  std::vector<double> stats(static_cast<size_t>(P) * P * 2);
+  std::vector<double> stats(static_cast<size_t>(P) * NG * 2);
   e = cudaMemcpyAsync(stats.data(), sums, stats.size() * sizeof(double), cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail(e, "anchor statistics copy");
   e = cudaStreamSynchronize(st);
@@ -627,10 +646,10 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
   const double rows = static_cast<double>(B) * H * n;
   for (int i = 0; i < P; ++i) {
     const double local_norm = std::sqrt(norms[i * 2 + 1]);
-    for (int j = 0; j < P; ++j) {
-      if (!sel.v[i * P + j]) continue;
-      pl->w[i * P + j] = stats[(i * P + j) * 2 + 0] / rows;
-      pl->alpha[i * P + j] = local_norm > 0.0 ? std::sqrt(stats[(i * P + j) * 2 + 1]) / local_norm : 0.0;
+    for (int G = 0; G < NG; ++G) {
+      if (!sel.v[i * NG + G]) continue;
+      pl->w[i * NG + G] = stats[(i * NG + G) * 2 + 0] / rows;
+      pl->alpha[i * NG + G] = local_norm > 0.0 ? std::sqrt(stats[(i * NG + G) * 2 + 1]) / local_norm : 0.0;
     }
   }
   pl->has_anchor = 1;

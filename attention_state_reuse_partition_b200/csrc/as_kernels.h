@@ -71,7 +71,7 @@ struct ComposePlan {
   float* lse;
 };
 
-// pair selection for the planner's anchor statistics ([P][P], 1 = reduce)
+// entry selection for the planner's anchor statistics ([P][n_groups], 1 = reduce)
 struct PlanRows {
   uint8_t v[AS_MAX_P * AS_MAX_P];
 };
@@ -82,8 +82,8 @@ cudaError_t launch_drift(const float* now, const float* anchor, int BH, int S, i
                          double* sums, cudaStream_t st);
 // address (on the current device) and size of the fixed drift scratch
 cudaError_t static_drift_scratch(double** ptr, size_t* capacity_doubles);
-cudaError_t launch_anchor_stats(const float* cache_out, const float* cache_lse, const float* lse_full,
-                                long long plane_out, long long plane_lse, int P, int BH, int S, int d,
+cudaError_t launch_anchor_stats(const void* cache_out, bool out_bf16, const float* cache_lse, const float* lse_full,
+                                long long plane_out, long long plane_lse, int P, int NG, int BH, int S, int d,
                                 const PlanRows& sel, double* partials, double* sums, cudaStream_t st);
 cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st);
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st);

@@ -63,17 +63,19 @@ __global__ void __launch_bounds__(THREADS) drift_partials_kernel(const float* __
   }
 }
 
-// partials[((i * P + j) * BH + bh) * 2 + {0, 1}] for selected pairs
-__global__ void __launch_bounds__(THREADS) stats_partials_kernel(const float* __restrict__ cache_out,
+// partials[((i * NG + G) * BH + bh) * 2 + {0, 1}] for selected entries (i, G);
+// OUT entries in fp32 or bf16 (OutT)
+template <class OutT>
+__global__ void __launch_bounds__(THREADS) stats_partials_kernel(const OutT* __restrict__ cache_out,
                                                                  const float* __restrict__ cache_lse,
                                                                  const float* __restrict__ lse_full,
-                                                                 long long plane_out, long long plane_lse, int P,
+                                                                 long long plane_out, long long plane_lse, int NG,
                                                                  int BH, int S, int d, int n,
                                                                  const __grid_constant__ PlanRows sel,
                                                                  double* __restrict__ partials) {
   __shared__ double sh[THREADS / 32];
   const int pair = blockIdx.x, bh = blockIdx.y;
-  const int i = pair / P, j = pair % P;
+  const int i = pair / NG, j = pair % NG;  // j: the entry's plane (its group)
   if (!sel.v[pair]) {
     if (threadIdx.x == 0) {
       partials[(static_cast<long long>(pair) * BH + bh) * 2 + 0] = 0.0;
@@ -84,12 +86,12 @@ __global__ void __launch_bounds__(THREADS) stats_partials_kernel(const float* __
   const long long row0 = static_cast<long long>(bh) * S + static_cast<long long>(i) * n;
   const float* lse_ij = cache_lse + j * plane_lse + row0;
   const float* lse_i = lse_full + row0;
-  const float* out_ij = cache_out + j * plane_out + row0 * d;
+  const OutT* out_ij = cache_out + j * plane_out + row0 * d;
   double ws = 0.0, sq = 0.0;
   for (int r = threadIdx.x; r < n; r += THREADS) ws += exp(static_cast<double>(lse_ij[r]) - lse_i[r]);
   const long long count = static_cast<long long>(n) * d;
   for (long long e = threadIdx.x; e < count; e += THREADS) {
-    const double o = out_ij[e];
+    const double o = static_cast<float>(out_ij[e]);
     sq += o * o;
   }
   const double sws = block_sum(ws, sh);
@@ -149,15 +151,21 @@ cudaError_t static_drift_scratch(double** ptr, size_t* capacity_doubles) {
   return cudaSuccess;
 }
 
-cudaError_t launch_anchor_stats(const float* cache_out, const float* cache_lse, const float* lse_full,
-                                long long plane_out, long long plane_lse, int P, int BH, int S, int d,
+cudaError_t launch_anchor_stats(const void* cache_out, bool out_bf16, const float* cache_lse, const float* lse_full,
+                                long long plane_out, long long plane_lse, int P, int NG, int BH, int S, int d,
                                 const PlanRows& sel, double* partials, double* sums, cudaStream_t st) {
   const int n = S / P;
-  stats_partials_kernel<<<dim3(P * P, BH), THREADS, 0, st>>>(cache_out, cache_lse, lse_full, plane_out, plane_lse,
-                                                              P, BH, S, d, n, sel, partials);
+  if (out_bf16)
+    stats_partials_kernel<__nv_bfloat16><<<dim3(P * NG, BH), THREADS, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(cache_out), cache_lse, lse_full, plane_out, plane_lse, NG, BH, S, d, n, sel,
+        partials);
+  else
+    stats_partials_kernel<float><<<dim3(P * NG, BH), THREADS, 0, st>>>(
+        static_cast<const float*>(cache_out), cache_lse, lse_full, plane_out, plane_lse, NG, BH, S, d, n, sel,
+        partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  sum_over_heads_kernel<<<(P * P + 127) / 128, 128, 0, st>>>(partials, P * P, BH, sums);
+  sum_over_heads_kernel<<<(P * NG + 127) / 128, 128, 0, st>>>(partials, P * NG, BH, sums);
   return cudaGetLastError();
 }
 

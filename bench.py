@@ -421,14 +421,15 @@ def run_video_long(args, device, g=1, cache_dtype="f32"):
             "steps": per_step, "reuse_mse_vs_full_last_step": mse}
 
 
-def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5):
+def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cache_dtype="f32"):
     """Long video trajectory with the anchor-guided planner choosing each
     step's plan: local states, drift, selection, the step, and the anchor
-    statistics after anchor steps."""
+    statistics after anchor steps.  With g > 1 the planner decides per cache
+    group of g KV partitions."""
     from attention_state_reuse_partition_b200 import api
     s = W.spec("video_long")
-    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
-    pl = api.AsPlanner(s.P, window, reuse_ratio, eps_local, s.B, s.H, s.S, s.d, device=device)
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, g=g, cache_dtype=cache_dtype)
+    pl = api.AsPlanner(s.P, window, reuse_ratio, eps_local, s.B, s.H, s.S, s.d, device=device, g=g)
     out = torch.empty((s.B, s.H, s.S, s.d), device=device)
     lse = torch.empty((s.B, s.H, s.S), device=device)
     local = torch.empty((s.B, s.H, s.S, s.d), device=device)
@@ -459,7 +460,9 @@ def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5):
     mse = torch.mean((out - full_o) ** 2).item()
     del cache, pl, full_o, out, lse, local, local_lse, last, q, k, v
     torch.cuda.empty_cache()
-    return {"workload": "video_long (4 steps) with the planner", "window": window, "reuse_ratio": reuse_ratio,
+    name = "video_long (4 steps) with the planner" if g == 1 else \
+        f"video_long (4 steps) with the planner over cache groups of {g} partitions, {cache_dtype} OUT entries"
+    return {"workload": name, "g": g, "cache_dtype": cache_dtype, "window": window, "reuse_ratio": reuse_ratio,
             "eps_local": eps_local, "steps": per_step, "reuse_mse_vs_full_last_step": mse,
             "timing": "wall clock around synchronising calls"}
 
@@ -473,7 +476,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
-    ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner"], default=None,
+    ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner",
+                                       "planner_grouped"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
@@ -494,7 +498,8 @@ def main():
     if args.only is not None:
         fn = {"compose": run_compose, "reuse": run_reuse, "video_long": run_video_long,
               "video_long_grouped": lambda a, dev: run_video_long(a, dev, g=4, cache_dtype="bf16"),
-              "planner": run_planner}[args.only]
+              "planner": run_planner,
+              "planner_grouped": lambda a, dev: run_planner(a, dev, g=4, cache_dtype="bf16")}[args.only]
         print(json.dumps({"only": args.only, **fn(args, device)}))
         return
     if world > 1:
@@ -514,6 +519,7 @@ def main():
         secondary["video_long"] = run_video_long(args, device)
         secondary["video_long_grouped"] = run_video_long(args, device, g=4, cache_dtype="bf16")
         secondary["planner"] = run_planner(args, device)
+        secondary["planner_grouped"] = run_planner(args, device, g=4, cache_dtype="bf16")
 
     cpu = None
     if rank == 0 and world == 1 and not args.kernel_only:

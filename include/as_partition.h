@@ -199,6 +199,13 @@ as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream);
  *   anchor     : when there is none yet, or max_i D(i,t)/||OUT_ta(i,i)||_F >
  *                eps_local; every pair fresh, every pair outside the window
  *                stored.
+ *   groups     : with cache groups of g partitions the planner decides per
+ *                group (Eq. 12, ASE of a group G_i): the unit (i, G) is the
+ *                set of G's members outside the window, w(i,G) and
+ *                alpha(i,G) come from its composed entry (w(i,G) is the sum of
+ *                its members' weights), the selection runs over the units,
+ *                and a unit's remote members are reused or stored together.
+ *                g = 1 is the per-pair planner.
  * A step with the planner:
  *   as_local_states(q,k,v,...) -> local_now            (device)
  *   as_planner_next(pl, local_now, local_anchor, ...)  -> plan, is_anchor
@@ -210,14 +217,20 @@ typedef struct as_planner {
   int P, window;
   double reuse_ratio, eps_local;
   int has_anchor;
-  double w[AS_MAX_P * AS_MAX_P];      /* w(i,j) of the last anchor (pairs outside the window) */
-  double alpha[AS_MAX_P * AS_MAX_P];  /* alpha(i,j) of the last anchor */
+  double w[AS_MAX_P * AS_MAX_P];      /* w(i,G) of the last anchor at [i*n_groups+G] */
+  double alpha[AS_MAX_P * AS_MAX_P];  /* alpha(i,G) of the last anchor */
   double drift[AS_MAX_P];             /* D(i,t) of the last as_planner_next (0 at anchors) */
   double rel_drift[AS_MAX_P];         /* D(i,t) / ||OUT_ta(i,i)||_F */
+  int g;                              /* cache group size the planner plans for */
 } as_planner;
 
-/* window >= 0, 0 <= reuse_ratio <= 1, eps_local >= 0, 1 <= P <= AS_MAX_P. */
+/* window >= 0, 0 <= reuse_ratio <= 1, eps_local >= 0, 1 <= P <= AS_MAX_P;
+ * per-pair planning (g = 1). */
 as_status as_planner_init(as_planner* pl, int P, int window, double reuse_ratio, double eps_local);
+
+/* As as_planner_init for a cache of groups of g partitions (1 <= g <= P);
+ * the cache passed to as_planner_commit_anchor must have the same g. */
+as_status as_planner_group_init(as_planner* pl, int P, int g, int window, double reuse_ratio, double eps_local);
 
 /* Bytes of device scratch the planner reductions need (8-byte aligned buffer,
  * caller-owned). */
@@ -260,20 +273,25 @@ as_status as_plan_drift_static(const float* now, const float* anchor, int B, int
 /* Host-only selection from ASE values h_ase [P*P] (see the readings above). */
 as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ratio, uint8_t* h_plan);
 
+/* The same per (i, G) unit for groups of g partitions: h_ase [P*n_groups]
+ * (entries of units without a remote member are ignored), h_plan [P*P]. */
+as_status as_plan_select_grouped(const double* h_ase, int P, int g, int window, double reuse_ratio,
+                                 uint8_t* h_plan);
+
 /* Plan of the next step.  local_now: the step's local states (as_local_states);
  * local_anchor [B,H,S,d]: the planner's copy of the anchor's local states,
  * overwritten (stream-ordered copy) when this step becomes an anchor.  Writes
- * h_plan [P*P], *h_is_anchor, and h_ase [P*P] (may be NULL; zeros at
+ * h_plan [P*P], *h_is_anchor, and h_ase [P*n_groups] (may be NULL; zeros at
  * anchors).  Synchronises `stream`. */
 as_status as_planner_next(as_planner* pl, const float* local_now, float* local_anchor, int B, int H, int S, int d,
                           void* scratch, size_t scratch_bytes, uint8_t* h_plan, int* h_is_anchor, double* h_ase,
                           void* stream);
 
 /* After an anchor step (the as_step that used the anchor plan h_plan):
- * measure w and alpha for every pair the plan stored, from the cache, the
- * step's composed LSE lse_full [B,H,S] and local_anchor.  Synchronises.
- * The cache must hold one fp32 entry per pair (g = 1, AS_F32), else
- * AS_ERR_UNSUPPORTED. */
+ * measure w and alpha for every entry (pair or group) the plan stored, from
+ * the cache (fp32 or bf16 entries), the step's composed LSE lse_full [B,H,S]
+ * and local_anchor.  The cache's group size must be the planner's
+ * (AS_ERR_INVALID_ARG otherwise).  Synchronises. */
 as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const float* lse_full,
                                    const float* local_anchor, const uint8_t* h_plan, void* scratch,
                                    size_t scratch_bytes, void* stream);

@@ -206,15 +206,38 @@ def test_plan_resolve_matches_oracle_on_random_plans(api):
             cache.set_member([[sum(1 << j for j in m) for m in row] for row in ocache.member])
 
 
-def test_planner_needs_a_pairwise_fp32_cache(api):
+def test_planner_and_cache_must_share_the_group_size(api):
+    """The anchor statistics read one entry per (i, G): a planner for groups
+    of g needs a cache of the same g (checked on the host, before any launch)."""
     from attention_state_reuse_partition_b200 import _lib
-    pl = api.AsPlanner(4, 1, 0.5, 0.1)
     plan = np.ones((4, 4), np.uint8)
-    for g, dt in [(2, "f32"), (1, "bf16")]:
-        cache = api.AsCache.host_only(1, 1, 64, 64, 4, g=g, cache_dtype=dt)
+    for pg, cg, dt in [(1, 2, "f32"), (2, 1, "bf16"), (4, 2, "bf16")]:
+        pl = api.AsPlanner(4, 1, 0.5, 0.1, g=pg)
+        cache = api.AsCache.host_only(1, 1, 64, 64, 4, g=cg, cache_dtype=dt)
         st = _lib.LIB.as_planner_commit_anchor(ctypes.byref(pl.struct), ctypes.byref(cache.struct), 1 << 20,
                                                1 << 20, plan.ctypes.data, 1 << 20, 1 << 30, None)
-        assert st == _lib.AS_ERR_UNSUPPORTED, (g, dt)
+        assert st == _lib.AS_ERR_INVALID_ARG, (pg, cg, dt)
+        assert "groups" in _lib.LIB.as_last_error().decode()
+
+
+def test_grouped_selection_matches_oracle(api):
+    """The C per-group selection against the hand-worked case and, bit-exactly,
+    the oracle's on random ASE values with ties, group sizes and windows."""
+    from oracle import as_oracle as O
+    a = np.array([[0.1, 0.5], [0.2, 0.9], [0.3, 0.05], [0.8, 0.4]])
+    want = np.array([[1, 0, 2, 2], [0, 1, 2, 2], [0, 0, 1, 0], [2, 2, 2, 1]], np.uint8)
+    assert np.array_equal(api.as_plan_select(a, 0, 0.5, g=2), want)
+    r = np.random.default_rng(8)
+    for trial in range(60):
+        P = int(r.integers(1, 24))
+        g = int(r.integers(1, P + 1))
+        window = int(r.integers(0, 4))
+        ase = np.round(r.random((P, (P + g - 1) // g)) * 4) / 4
+        ratio = float(r.choice([0.0, 0.25, 0.5, 0.9, 1.0, r.random()]))
+        assert np.array_equal(api.as_plan_select(ase, window, ratio, g=g), O.select_plan(ase, window, ratio, g)), \
+            (P, g, window, ratio)
+    with pytest.raises(api.AsError):
+        api.as_plan_select(np.zeros((4, 3)), 0, 0.5, g=2)
 
 
 def test_step_cache_miss_is_reported_before_any_launch(api):

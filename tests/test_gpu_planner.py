@@ -72,43 +72,57 @@ def test_drift_reduction(api):
         assert abs(drift[i] - rd) <= 1e-9 * rd and abs(norm[i] - rn) <= 1e-9 * rn
 
 
-def test_anchor_statistics(api):
+def _units(P, g, window):
+    """[P, n_groups] mask of the planner's units: groups with a member outside the window."""
+    NG = (P + g - 1) // g
+    return np.array([[any(abs(i - j) > window for j in range(G * g, min((G + 1) * g, P))) for G in range(NG)]
+                     for i in range(P)])
+
+
+@pytest.mark.parametrize("g,cache_dt", [(1, "f32"), (3, "f32"), (2, "bf16")])
+def test_anchor_statistics(api, g, cache_dt):
     """commit_anchor on a cache filled with known random states: w and alpha
-    of the stored pairs against float64 NumPy."""
+    of the stored entries (pairs, or groups of g) against float64 NumPy."""
     B, H, S, d, P, window = 1, 3, 8 * 64, 64, 8, 1
     n = S // P
-    cache = api.AsCache(B, H, S, d, P)
+    cache = api.AsCache(B, H, S, d, P, g=g, cache_dtype=cache_dt)
     outs, lses = cache.planes()
-    g = torch.Generator(device="cuda").manual_seed(12)
-    outs.copy_(torch.randn(outs.shape, generator=g, device="cuda"))
-    lses.copy_(torch.randn(lses.shape, generator=g, device="cuda") + 2.0)
-    lse_full = torch.randn((B, H, S), generator=g, device="cuda") + 4.0
-    pl = api.AsPlanner(P, window, 0.5, 0.1, B, H, S, d)
-    pl.local_anchor.copy_(torch.randn((B, H, S, d), generator=g, device="cuda"))
+    gen = torch.Generator(device="cuda").manual_seed(12)
+    outs.copy_(torch.randn(outs.shape, generator=gen, device="cuda"))
+    lses.copy_(torch.randn(lses.shape, generator=gen, device="cuda") + 2.0)
+    lse_full = torch.randn((B, H, S), generator=gen, device="cuda") + 4.0
+    pl = api.AsPlanner(P, window, 0.5, 0.1, B, H, S, d, g=g)
+    pl.local_anchor.copy_(torch.randn((B, H, S, d), generator=gen, device="cuda"))
     plan = O.anchor_plan(P, window)
     api.as_planner_commit_anchor(pl, cache, lse_full, plan)
     assert pl.has_anchor
     on, ln, lf, la = f64(outs), f64(lses), f64(lse_full), f64(pl.local_anchor)
+    units = _units(P, g, window)
     for i in range(P):
         local_norm = O.frob(la[..., i * n:(i + 1) * n, :])
-        for j in range(P):
-            if abs(i - j) <= window:
+        for G in range(units.shape[1]):
+            if not units[i, G]:
+                assert pl.w[i, G] == 0.0
                 continue
-            w_ref = float(np.mean(np.exp(ln[j][..., i * n:(i + 1) * n] - lf[..., i * n:(i + 1) * n])))
-            a_ref = O.frob(on[j][..., i * n:(i + 1) * n, :]) / local_norm
-            assert abs(pl.w[i, j] - w_ref) <= 1e-9 * w_ref, (i, j)
-            assert abs(pl.alpha[i, j] - a_ref) <= 1e-9 * a_ref, (i, j)
+            w_ref = float(np.mean(np.exp(ln[G][..., i * n:(i + 1) * n] - lf[..., i * n:(i + 1) * n])))
+            a_ref = O.frob(on[G][..., i * n:(i + 1) * n, :]) / local_norm
+            assert abs(pl.w[i, G] - w_ref) <= 1e-9 * w_ref, (i, G)
+            assert abs(pl.alpha[i, G] - a_ref) <= 1e-9 * a_ref, (i, G)
 
 
-def test_planner_trajectory_against_oracle(api):
+@pytest.mark.parametrize("g,cache_dt", [(1, "f32"), (4, "bf16")])
+def test_planner_trajectory_against_oracle(api, g, cache_dt):
     s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16, steps=6)
     P, n, window, ratio, eps_local = s.P, s.n, 2, 0.6, 0.25
     BAND = 1e-2
     steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
-    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P)
-    pl = api.AsPlanner(P, window, ratio, eps_local, s.B, s.H, s.S, s.d)
-    ocache = O.StateCache(P)
-    opl = O.Planner(P, window, ratio, eps_local)
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=g, cache_dtype=cache_dt)
+    pl = api.AsPlanner(P, window, ratio, eps_local, s.B, s.H, s.S, s.d, g=g)
+    ocache = O.StateCache(P, g, cache_dt)
+    opl = O.Planner(P, window, ratio, eps_local, g)
+    units = _units(P, g, window)
+    NG = units.shape[1]
+    member_of = np.array([[j // g for j in range(P)] for _ in range(P)])  # [i, j] -> G
     anchors = 0
     for t, (q, k, v) in enumerate(steps):
         qn, kn, vn = f64(q), f64(k), f64(v)
@@ -126,13 +140,15 @@ def test_planner_trajectory_against_oracle(api):
         if is_anchor != o_anchor:
             break  # an ambiguous anchor decision: the two trajectories part here
         if not is_anchor:
-            remote = np.abs(np.arange(P)[:, None] - np.arange(P)[None, :]) > window
-            vals = np.sort(oase[remote])
+            vals = np.sort(oase[units])
             k_reuse = int(np.floor(ratio * vals.size + 1e-9))
             thr = vals[k_reuse - 1] if k_reuse > 0 else -np.inf
-            ambiguous = remote & (np.abs(oase - thr) <= BAND * max(abs(thr), 1e-30))
+            amb_units = units & (np.abs(oase - thr) <= BAND * max(abs(thr), 1e-30))
+            ambiguous = np.take_along_axis(amb_units, member_of, axis=1)
             assert np.array_equal(plan[~ambiguous], oplan[~ambiguous]), f"plan at step {t}"
-            assert int((plan == O.PLAN_REUSE).sum()) == k_reuse
+            reused_units = sum(bool((plan[i, G * g:(G + 1) * g] == O.PLAN_REUSE).any())
+                               for i in range(P) for G in range(NG))
+            assert reused_units == k_reuse
         out, lse, hit, age = api.as_step(cache, q, k, v, plan, t)
         torch.cuda.synchronize()
         same_rows = [i for i in range(P) if np.array_equal(plan[i], oplan[i])]
@@ -144,9 +160,8 @@ def test_planner_trajectory_against_oracle(api):
             anchors += 1
             api.as_planner_commit_anchor(pl, cache, lse, plan)
             O.planner_commit_anchor(opl, ocache, ref_l, lambda i: np.arange(i * n, (i + 1) * n), n)
-            remote = np.abs(np.arange(P)[:, None] - np.arange(P)[None, :]) > window
-            assert np.allclose(pl.w[remote], opl.w[remote], rtol=5e-3, atol=0)
-            assert np.allclose(pl.alpha[remote], opl.alpha[remote], rtol=2e-2, atol=0)
+            assert np.allclose(pl.w[units], opl.w[units], rtol=5e-3, atol=0)
+            assert np.allclose(pl.alpha[units], opl.alpha[units], rtol=2e-2, atol=0)
         if len(same_rows) < P:
-            break  # plans differ on an ambiguous pair: the caches part here
+            break  # plans differ on an ambiguous unit: the caches part here
     assert anchors >= 1
