@@ -149,3 +149,28 @@ def test_step_grouped_video_long_full(api):
     assert cache.buffer.numel() == api.as_cache_bytes(s.B, s.H, s.S, s.d, s.P, 4, "bf16")
     del steps, cache
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("g,cache_dt,d,B", [(1, "f32", 64, 2), (3, "bf16", 128, 1), (8, "bf16", 64, 2)])
+def test_step_edge_plans(api, g, cache_dt, d, B):
+    """Rows with nothing fresh (every group reused), rows with no plain-fresh
+    partition (only stored groups, so no composite), a row of only fresh
+    pairs, and P at its maximum of 64 partitions for g = 8: the same
+    bookkeeping and states as the oracle over three steps."""
+    P = 64 if g == 8 else 6
+    n = 32 if P == 64 else 64
+    s = W.spec("flux_image", B=B, H=2, S=P * n, d=d, P=P)
+    steps = []
+    gen = torch.Generator(device="cuda").manual_seed(40 + g)
+    q, k, v = (x.cuda() for x in W.flux_qkv(s))
+    for t in range(3):
+        steps.append((q, (k.float() + 0.05 * t * torch.randn(k.shape, generator=gen, device="cuda")).to(k.dtype), v))
+    stored = np.full((P, P), W.PLAN_FRESH_STORE, np.uint8)
+    reuse = np.zeros((P, P), np.uint8)
+    reuse[1] = W.PLAN_FRESH            # a row of only fresh pairs
+    reuse[2] = W.PLAN_FRESH_STORE      # a row of only stored groups: no composite
+    reuse[3, 0:g] = W.PLAN_FRESH       # a row with one plain-fresh group, the rest reused
+    plans = [stored, reuse, reuse.copy()]
+    plans[2][2] = 0                    # row 2 reuses what step 1 stored
+    _run_grouped(api, s, steps, plans, g, cache_dt,
+                 dtype_check=check_bf16 if s.dtype == "bf16" else check_f32)
