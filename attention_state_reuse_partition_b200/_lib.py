@@ -24,7 +24,8 @@ EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as
            "as_cache_init", "as_plan_resolve", "as_step", "as_device_status", "as_debug_timeout_probe",
            "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
            "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static",
-           "as_cache_group_bytes", "as_cache_group_init", "as_planner_group_init", "as_plan_select_grouped")
+           "as_cache_group_bytes", "as_cache_group_init", "as_planner_group_init", "as_plan_select_grouped",
+           "as_step_local")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -90,6 +91,9 @@ def _load() -> ctypes.CDLL:
     lib.as_step.restype = c_int
     lib.as_step.argtypes = [ctypes.POINTER(AsCacheStruct), vp, vp, vp, c_int, c_float, vp, c_int, vp, vp,
                             vp, vp, vp]
+    lib.as_step_local.restype = c_int
+    lib.as_step_local.argtypes = [ctypes.POINTER(AsCacheStruct), vp, vp, vp, c_int, c_float, vp, c_int, vp, vp,
+                                  vp, vp, vp, vp, vp]
     lib.as_device_status.restype = c_int
     lib.as_device_status.argtypes = [vp, ctypes.POINTER(u32)]
     lib.as_debug_timeout_probe.restype = c_int

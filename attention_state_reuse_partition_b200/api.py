@@ -18,7 +18,7 @@ __all__ = ["as_partition_attn", "as_compose", "as_cache_bytes", "as_cache_init",
            "as_device_status", "as_debug_timeout_probe", "as_version", "AsCache", "AsError",
            "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE", "AsPlanner", "as_planner_init",
            "as_planner_scratch_bytes", "as_local_states", "as_plan_drift", "as_plan_select", "as_planner_next",
-           "as_planner_commit_anchor", "as_plan_drift_static"]
+           "as_planner_commit_anchor", "as_plan_drift_static", "as_step_local"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -198,6 +198,28 @@ def as_step(cache: AsCache, q, k, v, plan, step: int, scale: Optional[float] = N
     check(LIB.as_step(ctypes.byref(cache.struct), _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q),
                       float(scale), arr.ctypes.data, int(step), _dev(out, "out"), _dev(lse, "lse"),
                       hit.ctypes.data, age.ctypes.data, _stream_ptr(stream)))
+    return out, lse, hit.reshape(P, P), age.reshape(P, P)
+
+
+def as_step_local(cache: AsCache, q, k, v, plan, step: int, local_out, local_lse, scale: Optional[float] = None,
+                  out=None, lse=None, stream=None):
+    """as_step with the step's local states AS(i, i) given (from
+    as_local_states on the same inputs): plain-fresh diagonal pairs are
+    composed from them instead of recomputed.  Returns (out, lse, hit, age)."""
+    B, H, S, d = q.shape
+    P = cache.P
+    scale = 1.0 / d ** 0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, S, d), device=q.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    arr = _plan_bytes(plan, P)
+    hit = np.zeros(P * P, dtype=np.uint8)
+    age = np.zeros(P * P, dtype=np.int32)
+    check(LIB.as_step_local(ctypes.byref(cache.struct), _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q),
+                            float(scale), arr.ctypes.data, int(step), _dev(local_out, "local_out"),
+                            _dev(local_lse, "local_lse"), _dev(out, "out"), _dev(lse, "lse"), hit.ctypes.data,
+                            age.ctypes.data, _stream_ptr(stream)))
     return out, lse, hit.reshape(P, P), age.reshape(P, P)
 
 

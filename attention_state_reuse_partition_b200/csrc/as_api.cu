@@ -323,15 +323,18 @@ as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step, ui
   return ok();
 }
 
-as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
-                  const uint8_t* h_plan, int step, float* out, float* lse, uint8_t* h_hit, int32_t* h_age,
-                  void* stream) {
+// as_step and as_step_local; local_out == nullptr: no precomputed local states
+static as_status step_impl(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
+                           const uint8_t* h_plan, int step, const float* local_out, const float* local_lse,
+                           float* out, float* lse, uint8_t* h_hit, int32_t* h_age, void* stream) {
   as_status s = check_cache(c);
   if (s != AS_OK) return s;
   if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
   if (!q || !k || !v || !out || !lse || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(AS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (local_out && (!local_lse || !aligned16(local_out) || !aligned16(local_lse)))
+    return fail(AS_ERR_INVALID_ARG, "local states must be non-null and 16-byte aligned");
   if (!(scale > 0.f)) return fail(AS_ERR_INVALID_ARG, "scale must be > 0");
   const int B = c->B, H = c->H, S = c->S, d = c->d, P = c->P, n = S / P, g = c->g, NG = c->n_groups;
   uint8_t hit[AS_MAX_P * AS_MAX_P];
@@ -339,6 +342,8 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   if ((s = resolve(c, h_plan, step, hit, age)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // a plain-fresh diagonal pair whose state the caller already holds
+  auto local_of = [&](int i) { return local_out != nullptr && h_plan[i * P + i] == AS_PLAN_FRESH; };
 
   // fresh pairs: composite of the plain-fresh partitions -> out/lse; the
   // stored members of each group -> one composed state in the group's plane
@@ -347,21 +352,21 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   L.n_blocks = P;
   L.block_rows = n;
   L.block_row0 = 0;
-  bool any_fresh = false, need_compose = false;
+  bool any_fresh = false;
   for (int i = 0; i < P; ++i) {
     for (int j = 0; j < P; ++j) {
       const uint8_t pc = h_plan[i * P + j];
-      L.code[i * P + j] = pc == AS_PLAN_FRESH ? AS_KCODE_COMPOSE : pc == AS_PLAN_FRESH_STORE ? AS_KCODE_EMIT
-                                                                                            : AS_KCODE_SKIP;
-      any_fresh |= pc != AS_PLAN_REUSE;
-      need_compose |= pc != AS_PLAN_FRESH;
+      uint8_t kc = pc == AS_PLAN_FRESH ? AS_KCODE_COMPOSE : pc == AS_PLAN_FRESH_STORE ? AS_KCODE_EMIT : AS_KCODE_SKIP;
+      if (j == i && local_of(i)) kc = AS_KCODE_SKIP;
+      L.code[i * P + j] = kc;
+      any_fresh |= kc != AS_KCODE_SKIP;
     }
   }
   for (int j = 0; j < P; ++j) L.dest_of[j] = static_cast<int8_t>(j / g);
   // every query partition reads the same KV list: one block of S rows, so
   // query tiles are not cut at partition boundaries
   bool uniform = true;
-  for (int i = 1; i < P && uniform; ++i) uniform = std::memcmp(h_plan, h_plan + i * P, P) == 0;
+  for (int i = 1; i < P && uniform; ++i) uniform = std::memcmp(L.code, L.code + i * P, P) == 0;
   if (uniform) {
     L.n_blocks = 1;
     L.block_rows = S;
@@ -379,38 +384,37 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   L.dst_plane_lse = static_cast<long long>(B) * H * S;
   if (any_fresh && (s = launch_attn(L, dt, st)) != AS_OK) return s;
 
-  // final composition: composite + stored group entries + reused group entries
+  // final composition: composite + local state + stored and reused group entries
+  asp::ComposePlan a;
+  std::memset(&a, 0, sizeof(a));
+  bool need_compose = false;
+  for (int i = 0; i < P; ++i) {
+    int cnt = 0;
+    bool composite = false;
+    for (int j = 0; j < P; ++j) composite |= L.code[i * P + j] == AS_KCODE_COMPOSE;
+    if (composite) a.src[i][cnt++] = -1;
+    if (local_of(i)) a.src[i][cnt++] = -2;
+    for (int G = 0; G < NG; ++G)
+      if (group_mask(h_plan, P, g, i, G, AS_PLAN_REUSE) || group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE))
+        a.src[i][cnt++] = static_cast<int8_t>(G);
+    // a row whose only source is the composite already holds its final state
+    a.nsrc[i] = (cnt == 1 && composite) ? 0 : static_cast<uint8_t>(cnt);
+    need_compose |= a.nsrc[i] > 0;
+  }
   if (need_compose) {
-    asp::ComposePlan a;
-    std::memset(&a, 0, sizeof(a));
     a.B = B;
     a.H = H;
     a.S = S;
     a.d = d;
     a.P = P;
     a.n = n;
-    for (int i = 0; i < P; ++i) {
-      int cnt = 0;
-      bool has_fresh = false, has_other = false;
-      for (int j = 0; j < P; ++j) {
-        has_fresh |= h_plan[i * P + j] == AS_PLAN_FRESH;
-        has_other |= h_plan[i * P + j] != AS_PLAN_FRESH;
-      }
-      if (!has_other) {
-        a.nsrc[i] = 0;  // the composite already is the final state
-        continue;
-      }
-      if (has_fresh) a.src[i][cnt++] = -1;
-      for (int G = 0; G < NG; ++G)
-        if (group_mask(h_plan, P, g, i, G, AS_PLAN_REUSE) || group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE))
-          a.src[i][cnt++] = static_cast<int8_t>(G);
-      a.nsrc[i] = static_cast<uint8_t>(cnt);
-    }
     a.cache_out = c->out_planes;
     a.cache_bf16 = c->cache_dt == AS_BF16;
     a.cache_lse = c->lse_planes;
     a.plane_out = L.dst_plane_out;
     a.plane_lse = L.dst_plane_lse;
+    a.local_out = local_out;
+    a.local_lse = local_lse;
     a.out = out;
     a.lse = lse;
     cudaError_t e = asp::launch_compose_plan(a, st);
@@ -427,6 +431,19 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
   if (h_hit) std::memcpy(h_hit, hit, static_cast<size_t>(P) * P);
   if (h_age) std::memcpy(h_age, age, static_cast<size_t>(P) * P * sizeof(int32_t));
   return ok();
+}
+
+as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
+                  const uint8_t* h_plan, int step, float* out, float* lse, uint8_t* h_hit, int32_t* h_age,
+                  void* stream) {
+  return step_impl(c, q, k, v, dt, scale, h_plan, step, nullptr, nullptr, out, lse, h_hit, h_age, stream);
+}
+
+as_status as_step_local(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
+                        const uint8_t* h_plan, int step, const float* local_out, const float* local_lse, float* out,
+                        float* lse, uint8_t* h_hit, int32_t* h_age, void* stream) {
+  if (!local_out || !local_lse) return fail(AS_ERR_INVALID_ARG, "null local states");
+  return step_impl(c, q, k, v, dt, scale, h_plan, step, local_out, local_lse, out, lse, h_hit, h_age, stream);
 }
 
 as_status as_device_status(void* stream, uint32_t* h_bits) {

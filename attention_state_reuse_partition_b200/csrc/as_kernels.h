@@ -61,12 +61,15 @@ struct ComposeStrided {
 // query partition from the step plan
 struct ComposePlan {
   int B, H, S, d, P, n;
-  int8_t src[AS_MAX_P][AS_MAX_P + 1];  // per query partition: -1 = composite, G = cache plane G
+  // per query partition: -1 = composite, -2 = local state, G = cache plane G
+  int8_t src[AS_MAX_P][AS_MAX_P + 2];
   uint8_t nsrc[AS_MAX_P];
   const void* cache_out;  // fp32, or bf16 when cache_bf16
   int cache_bf16;
   const float* cache_lse;
   long long plane_out, plane_lse;
+  const float* local_out;  // [B,H,S,d] local states AS(i,i) (source -2), may be null
+  const float* local_lse;
   float* out;  // [B,H,S,d]: holds the composite on entry (where used), the final state on exit
   float* lse;
 };

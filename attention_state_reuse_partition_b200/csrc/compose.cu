@@ -198,7 +198,8 @@ __global__ void __launch_bounds__(WARPS * 32) compose_plan_kernel(const __grid_c
     const int8_t* list = a.src[i];
     auto src = [&](int k) {
       const int j = list[k];
-      if (j < 0) return Ptrs{a.out, a.lse, false};
+      if (j == -1) return Ptrs{a.out, a.lse, false};
+      if (j == -2) return Ptrs{a.local_out, a.local_lse, false};
       if (a.cache_bf16)
         return Ptrs{static_cast<const __nv_bfloat16*>(a.cache_out) + j * a.plane_out, a.cache_lse + j * a.plane_lse, true};
       return Ptrs{static_cast<const float*>(a.cache_out) + j * a.plane_out, a.cache_lse + j * a.plane_lse, false};

@@ -423,7 +423,8 @@ def run_video_long(args, device, g=1, cache_dtype="f32"):
 
 def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cache_dtype="f32"):
     """Long video trajectory with the anchor-guided planner choosing each
-    step's plan: local states, drift, selection, the step, and the anchor
+    step's plan: local states, drift, selection, the step (which composes the
+    local states instead of recomputing the diagonal pairs), and the anchor
     statistics after anchor steps.  With g > 1 the planner decides per cache
     group of g KV partitions."""
     from attention_state_reuse_partition_b200 import api
@@ -442,7 +443,7 @@ def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cac
         api.as_local_states(q, k, v, s.P, out=local, lse=local_lse)
         plan, is_anchor, _ = api.as_planner_next(pl, local)          # synchronises
         t1 = time.perf_counter()
-        api.as_step(cache, q, k, v, plan, t, out=out, lse=lse)
+        api.as_step_local(cache, q, k, v, plan, t, local, local_lse, out=out, lse=lse)
         torch.cuda.synchronize()
         t2 = time.perf_counter()
         if is_anchor:

@@ -173,6 +173,19 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
                   const uint8_t* h_plan, int step, float* out, float* lse,
                   uint8_t* h_hit, int32_t* h_age, void* stream);
 
+/* as_step for a caller that already holds the step's local states
+ * AS_step(i,i) (as_local_states on the same q, k, v and scale, which the
+ * anchor-guided planner computes every step to measure its drift).  Every
+ * diagonal pair the plan marks AS_PLAN_FRESH is composed from local_out
+ * [B,H,S,d] / local_lse [B,H,S] (fp32, device, 16-byte aligned) instead of
+ * being recomputed; everything else is as_step's.  The review page
+ * ("Circularity Check", on Eq. 10) describes the local state as the one
+ * computed at every step; this entry point keeps it from being computed
+ * twice. */
+as_status as_step_local(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
+                        const uint8_t* h_plan, int step, const float* local_out, const float* local_lse,
+                        float* out, float* lse, uint8_t* h_hit, int32_t* h_age, void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word that the
  * kernels' bounded waits set.  *h_bits receives the raw bits (may be NULL).
  * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, else AS_OK. */

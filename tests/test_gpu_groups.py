@@ -174,3 +174,34 @@ def test_step_edge_plans(api, g, cache_dt, d, B):
     plans[2][2] = 0                    # row 2 reuses what step 1 stored
     _run_grouped(api, s, steps, plans, g, cache_dt,
                  dtype_check=check_bf16 if s.dtype == "bf16" else check_f32)
+
+
+@pytest.mark.parametrize("g,cache_dt", [(1, "f32"), (4, "bf16")])
+def test_step_local_reuses_the_local_states(api, g, cache_dt):
+    """as_step_local with the step's local states from as_local_states: the
+    same bookkeeping and, within the parity tolerances, the same states as
+    the oracle and as as_step (which recomputes the diagonal pairs).  The
+    plans also hold rows whose diagonal is stored or reused, where the local
+    states are not used."""
+    s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16)
+    steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
+    plans = [W.grouped_plan_for_step(s, t, g).numpy() for t in range(s.steps)]
+    plans[1][0, :] = W.PLAN_FRESH_STORE   # row 0 stores everything, its diagonal included
+    plans[2][0, :] = W.PLAN_REUSE         # ... and reuses exactly those entries afterwards
+    plans[3][0, :] = W.PLAN_REUSE
+    ca = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=g, cache_dtype=cache_dt)
+    cb = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=g, cache_dtype=cache_dt)
+    ocache = O.StateCache(s.P, g, cache_dt)
+    for t, (q, k, v) in enumerate(steps):
+        plan = plans[t]
+        lo, ll = api.as_local_states(q, k, v, s.P)
+        out, lse, hit, age = api.as_step_local(ca, q, k, v, plan, t, lo, ll)
+        out_b, lse_b, hit_b, age_b = api.as_step(cb, q, k, v, plan, t)
+        torch.cuda.synchronize()
+        ref_o, ref_l, ref_hit, ref_age = O.step(ocache, f64(q), f64(k), f64(v), plan, t, s.scale)
+        assert np.array_equal(hit, ref_hit) and np.array_equal(age, ref_age), t
+        assert np.array_equal(hit, hit_b) and np.array_equal(ca.t_c, cb.t_c) and np.array_equal(ca.member, cb.member)
+        check_bf16(out, lse, ref_o, ref_l, f"as_step_local g={g} step {t}")
+        # the two differ where P is rounded to bf16: against the diagonal's own
+        # running maximum here, against the whole window's in as_step
+        check_bf16(out, lse, f64(out_b), f64(lse_b), f"as_step_local vs as_step g={g} step {t}")
