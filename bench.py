@@ -267,36 +267,65 @@ def run_own(args, rank, world, device):
     if args.kernel_only:
         return result, (q, k, v, s)
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers.  Steps are
+    # independent, so they are pipelined over three streams with two buffer
+    # sets: the host->device copy of step i+1 and the device->host copy of
+    # step i-1 overlap the attention of step i (PCIe is full duplex).  Every
+    # step still copies its inputs in and its result out inside the timed
+    # region.
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
-    hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    NB = 2
+    hout = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(NB)]
+    hlse = [torch.empty(lse.shape, dtype=torch.float32).pin_memory() for _ in range(NB)]
+    din = [tuple(torch.empty_like(x) for x in (q, k, v)) for _ in range(NB)]
+    dout = [(torch.empty_like(out), torch.empty_like(lse)) for _ in range(NB)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(NB)]
+    ev_cmp = [torch.cuda.Event() for _ in range(NB)]
+    ev_out = [torch.cuda.Event() for _ in range(NB)]
+    for b in range(NB):  # nothing in flight yet
+        ev_cmp[b].record(s_cmp)
+        ev_out[b].record(s_out)
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        api.as_step(cache, dq, dk, dv, plan, 0, out=out, lse=lse)
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+    def e2e_step(i):
+        b = i % NB
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[b])             # the step that last read din[b] is done
+            for dst, src in zip(din[b], (hq, hk, hv)):
+                dst.copy_(src, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            s_cmp.wait_event(ev_out[b])            # dout[b] has been copied out
+            api.as_step(cache, *din[b], plan, 0, out=dout[b][0], lse=dout[b][1], stream=s_cmp)
+            ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            hout[b].copy_(dout[b][0], non_blocking=True)
+            hlse[b].copy_(dout[b][1], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(args.steps):
+        e2e_step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
-    d2h = hout.numel() * 4 + hlse.numel() * 4
-    assert torch.allclose(hout.to(device), out), "e2e output differs from the device-resident run"
+    d2h = hout[0].numel() * 4 + hlse[0].numel() * 4
+    for b in range(NB):
+        assert torch.allclose(hout[b].to(device), out), "e2e output differs from the device-resident run"
 
     result["e2e"] = {"value": weak_scaling_value(flops, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
-                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                     "pipeline": "3 streams, 2 buffer sets: copy-in, attention and copy-out of consecutive "
+                                 "steps overlap"}
     del cache, flush
     torch.cuda.empty_cache()
     return result, (q, k, v, s)
