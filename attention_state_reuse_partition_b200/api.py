@@ -150,6 +150,27 @@ class AsCache:
     def member(self) -> np.ndarray:
         return np.ctypeslib.as_array(self.struct.member)[: self.P * self.NG].reshape(self.P, self.NG).copy()
 
+    def state_dict(self) -> dict:
+        """Everything needed to resume: sizes, group size, entry dtype, the
+        host bookkeeping (t_c, member masks) and a host copy of the device
+        buffer (synchronises the current stream)."""
+        return {"sizes": (self.B, self.H, self.S, self.d, self.P), "g": self.g,
+                "cache_dtype": "bf16" if self.cache_dtype == torch.bfloat16 else "f32",
+                "t_c": self.t_c, "member": self.member,
+                "buffer": None if self.buffer is None else self.buffer.cpu()}
+
+    @classmethod
+    def from_state_dict(cls, sd: dict, device="cuda") -> "AsCache":
+        """A cache restored from state_dict(): same entries and bookkeeping."""
+        B, H, S, d, P = sd["sizes"]
+        self = cls(B, H, S, d, P, device=device, g=sd["g"], cache_dtype=sd["cache_dtype"])
+        if sd["buffer"] is None or sd["buffer"].numel() != self.buffer.numel():
+            raise AsError(_lib.AS_ERR_INVALID_ARG, "state dict buffer does not match the cache sizes")
+        self.buffer.copy_(sd["buffer"])
+        self.set_t_c(sd["t_c"])
+        self.set_member(sd["member"])
+        return self
+
     def planes(self):
         """Views of the cache planes: OUT [NG,B,H,S,d] (the cache dtype), LSE
         [NG,B,H,S] (fp32)."""

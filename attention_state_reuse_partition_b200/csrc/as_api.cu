@@ -14,6 +14,8 @@
 #include <tuple>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "as_kernels.h"
 #include "as_partition.h"
 
@@ -37,6 +39,13 @@ as_status ok() {
   g_err.clear();
   return AS_OK;
 }
+
+// NVTX range around an entry point, so that profiler timelines show each call
+// (a no-op unless a tool is attached)
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
 
 as_status cuda_fail(cudaError_t e, const char* what) {
   return fail(AS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -204,6 +213,7 @@ const char* as_version(void) { return "attention-state-reuse-partition b200 0.1 
 as_status as_partition_attn(const void* q, const void* k, const void* v, as_dtype dt, int B, int H, int S, int d,
                             int P, float scale, int q_part, const int32_t* h_kv_parts, int n_kv_parts, int compose,
                             float* out, float* lse, void* stream) {
+  Range nvtx_range("as_partition_attn");
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
@@ -245,6 +255,7 @@ as_status as_partition_attn(const void* q, const void* k, const void* v, as_dtyp
 
 as_status as_compose(const float* outs, const float* lses, int n_states, int64_t rows, int d,
                      int64_t state_stride_out, int64_t state_stride_lse, float* out, float* lse, void* stream) {
+  Range nvtx_range("as_compose");
   if (d != 64 && d != 128) return fail(AS_ERR_INVALID_ARG, "d must be 64 or 128 (got %d)", d);
   if (n_states < 1) return fail(AS_ERR_INVALID_ARG, "n_states must be >= 1");
   if (rows < 0) return fail(AS_ERR_INVALID_ARG, "rows must be >= 0");
@@ -327,6 +338,7 @@ as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step, ui
 static as_status step_impl(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
                            const uint8_t* h_plan, int step, const float* local_out, const float* local_lse,
                            float* out, float* lse, uint8_t* h_hit, int32_t* h_age, void* stream) {
+  Range nvtx_range(local_out ? "as_step_local" : "as_step");
   as_status s = check_cache(c);
   if (s != AS_OK) return s;
   if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
@@ -491,6 +503,7 @@ size_t as_planner_scratch_bytes(int B, int H, int P) {
 
 as_status as_local_states(const void* q, const void* k, const void* v, as_dtype dt, int B, int H, int S, int d,
                           int P, float scale, float* out, float* lse, void* stream) {
+  Range nvtx_range("as_local_states");
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
@@ -519,6 +532,7 @@ as_status as_local_states(const void* q, const void* k, const void* v, as_dtype 
 
 as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int S, int d, int P, void* scratch,
                         size_t scratch_bytes, double* h_drift, double* h_norm, void* stream) {
+  Range nvtx_range("as_plan_drift");
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (!now || !anchor || !h_drift || !h_norm) return fail(AS_ERR_INVALID_ARG, "null pointer");
@@ -536,6 +550,7 @@ as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int
 
 as_status as_plan_drift_static(const float* now, const float* anchor, int B, int H, int S, int d, int P,
                                double* h_drift, double* h_norm, void* stream) {
+  Range nvtx_range("as_plan_drift_static");
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (!now || !anchor || !h_drift || !h_norm) return fail(AS_ERR_INVALID_ARG, "null pointer");
@@ -585,6 +600,7 @@ as_status as_plan_select(const double* h_ase, int P, int window, double reuse_ra
 as_status as_planner_next(as_planner* pl, const float* local_now, float* local_anchor, int B, int H, int S, int d,
                           void* scratch, size_t scratch_bytes, uint8_t* h_plan, int* h_is_anchor, double* h_ase,
                           void* stream) {
+  Range nvtx_range("as_planner_next");
   as_status s = check_planner(pl);
   if (s != AS_OK) return s;
   const int P = pl->P;
@@ -628,6 +644,7 @@ as_status as_planner_next(as_planner* pl, const float* local_now, float* local_a
 as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const float* lse_full,
                                    const float* local_anchor, const uint8_t* h_plan, void* scratch,
                                    size_t scratch_bytes, void* stream) {
+  Range nvtx_range("as_planner_commit_anchor");
   as_status s = check_planner(pl);
   if (s != AS_OK) return s;
   if ((s = check_cache(c)) != AS_OK) return s;

@@ -282,3 +282,19 @@ def test_planner_init_validation(api):
     pl = api.AsPlanner(8, 2, 0.6, 0.05)
     assert not pl.has_anchor and pl.P == 8
     assert api.as_planner_scratch_bytes(1, 40, 32) == (32 * 32 * 40 * 2 + 32 * 32 * 2) * 8
+
+
+def test_cache_bookkeeping_round_trip(api):
+    """The host bookkeeping of a cache survives state_dict (no device buffer
+    on a machine without a GPU)."""
+    cache = api.AsCache.host_only(1, 1, 64, 64, 8, g=3, cache_dtype="bf16")
+    t_c = np.arange(8 * 3).reshape(8, 3) - 5
+    member = np.arange(8 * 3, dtype=np.uint64).reshape(8, 3) * 7
+    cache.set_t_c(t_c)
+    cache.set_member(member)
+    sd = cache.state_dict()
+    assert sd["g"] == 3 and sd["cache_dtype"] == "bf16" and sd["buffer"] is None
+    other = api.AsCache.host_only(1, 1, 64, 64, 8, g=3, cache_dtype="bf16")
+    other.set_t_c(sd["t_c"])
+    other.set_member(sd["member"])
+    assert np.array_equal(other.t_c, t_c) and np.array_equal(other.member, member)

@@ -205,3 +205,24 @@ def test_step_local_reuses_the_local_states(api, g, cache_dt):
         # the two differ where P is rounded to bf16: against the diagonal's own
         # running maximum here, against the whole window's in as_step
         check_bf16(out, lse, f64(out_b), f64(lse_b), f"as_step_local vs as_step g={g} step {t}")
+
+
+def test_cache_checkpoint_and_resume(api, tmp_path):
+    """A cache saved after the anchor step (torch.save of state_dict) and
+    restored into a new buffer gives bit-identical reuse steps."""
+    s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16)
+    steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
+    plans = [W.grouped_plan_for_step(s, t, 4).numpy() for t in range(s.steps)]
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=4, cache_dtype="bf16")
+    api.as_step(cache, *steps[0], plans[0], 0)
+    torch.cuda.synchronize()
+    path = tmp_path / "cache.pt"
+    torch.save(cache.state_dict(), path)
+    restored = api.AsCache.from_state_dict(torch.load(path, weights_only=False))
+    assert np.array_equal(restored.t_c, cache.t_c) and np.array_equal(restored.member, cache.member)
+    for t in range(1, s.steps):
+        a = api.as_step(cache, *steps[t], plans[t], t)
+        b = api.as_step(restored, *steps[t], plans[t], t)
+        torch.cuda.synchronize()
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]), t
+        assert np.array_equal(a[2], b[2]) and np.array_equal(a[3], b[3])
