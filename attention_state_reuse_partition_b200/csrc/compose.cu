@@ -32,13 +32,15 @@ template <>
 struct Vec<128> {
   using T = float4;
   static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-  // this lane's 4 elements of row `row` of a fp32 or bf16 state
-  static __device__ __forceinline__ float4 load(const void* base, long long row, int lane, bool bf16) {
-    if (bf16) {
-      const uint2 u = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + row * 128)[lane];
+  // this lane's 4 elements of row `row` of a state stored as E (fp32 or bf16)
+  template <class E>
+  static __device__ __forceinline__ float4 load(const void* base, long long row, int lane) {
+    if constexpr (sizeof(E) == 2) {
+      const uint2 u = reinterpret_cast<const uint2*>(static_cast<const E*>(base) + row * 128)[lane];
       return make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
+    } else {
+      return reinterpret_cast<const float4*>(static_cast<const E*>(base) + row * 128)[lane];
     }
-    return reinterpret_cast<const float4*>(static_cast<const float*>(base) + row * 128)[lane];
   }
   static __device__ __forceinline__ void fma(float4& a, float c, const float4& x) {
     a.x = fmaf(c, x.x, a.x);
@@ -51,12 +53,14 @@ template <>
 struct Vec<64> {
   using T = float2;
   static __device__ __forceinline__ float2 zero() { return make_float2(0.f, 0.f); }
-  static __device__ __forceinline__ float2 load(const void* base, long long row, int lane, bool bf16) {
-    if (bf16) {
-      const uint32_t u = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(base) + row * 64)[lane];
+  template <class E>
+  static __device__ __forceinline__ float2 load(const void* base, long long row, int lane) {
+    if constexpr (sizeof(E) == 2) {
+      const uint32_t u = reinterpret_cast<const uint32_t*>(static_cast<const E*>(base) + row * 64)[lane];
       return make_float2(bf_lo(u), bf_hi(u));
+    } else {
+      return reinterpret_cast<const float2*>(static_cast<const E*>(base) + row * 64)[lane];
     }
-    return reinterpret_cast<const float2*>(static_cast<const float*>(base) + row * 64)[lane];
   }
   static __device__ __forceinline__ void fma(float2& a, float c, const float2& x) {
     a.x = fmaf(c, x.x, a.x);
@@ -78,15 +82,16 @@ __device__ __forceinline__ float warp_sum(float x) {
 struct Ptrs {
   const void* first;    // OUT base
   const float* second;  // LSE base
-  bool bf16;            // OUT in bf16
 };
 
 // Composes rows [row0, row0+nr) (nr <= RB) of `nsrc` sources.  src(k) gives the
 // base pointers (out_base, lse_base) of source k such that row r's state is at
-// row r of out_base (fp32, or bf16 when the source says so) and lse_base + r.  The output may alias a source: every source
-// row is read before the output row is written, by the same warp.
-template <int D, class SrcFn>
-__device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, SrcFn src, float* out,
+// row r of out_base and lse_base + r.  Sources [0, nf) keep OUT in fp32, the
+// others in E (fp32 or bf16), so that every batch of loads has one type.  The
+// output may alias a source: every source row is read before the output row
+// is written, by the same warp.
+template <int D, class E, class SrcFn>
+__device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, int nf, SrcFn src, float* out,
                                              float* lse, int lane) {
   using V = Vec<D>;
   using T = typename V::T;
@@ -135,25 +140,23 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, S
       for (int rr = 0; rr < RB; ++rr) coef[rr] = 0.f;
     }
     const int kn = min(32, nsrc - k0);
+    // one source at a time (its pointers resolved once), its rows' loads in
+    // flight together
+    for (int kk = 0; kk < kn; ++kk) {
+      const Ptrs sp = src(k0 + kk);
+      T x[RB];
+      if (k0 + kk < nf) {
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) {
-      if (rr >= nr) break;
-      int kk = 0;
-      for (; kk + 8 <= kn; kk += 8) {
-        T x[8];
+        for (int rr = 0; rr < RB; ++rr)
+          if (rr < nr) x[rr] = V::template load<float>(sp.first, row0 + rr, lane);
+      } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const Ptrs sp = src(k0 + kk + u);
-          x[u] = V::load(sp.first, row0 + rr, lane, sp.bf16);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk + u), x[u]);
+        for (int rr = 0; rr < RB; ++rr)
+          if (rr < nr) x[rr] = V::template load<E>(sp.first, row0 + rr, lane);
       }
-      for (; kk < kn; ++kk) {
-        const Ptrs sp = src(k0 + kk);
-        const T x = V::load(sp.first, row0 + rr, lane, sp.bf16);
-        V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk), x);
-      }
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr)
+        if (rr < nr) V::fma(acc[rr], __shfl_sync(0xffffffffu, coef[rr], kk), x[rr]);
     }
   }
 #pragma unroll
@@ -165,23 +168,24 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, S
 }
 
 template <int D>
-__global__ void __launch_bounds__(WARPS * 32) compose_strided_kernel(const __grid_constant__ ComposeStrided a) {
+__global__ void __launch_bounds__(WARPS * 32, 2) compose_strided_kernel(const __grid_constant__ ComposeStrided a) {
   const int lane = threadIdx.x & 31;
   const long long nblk = (a.rows + RB - 1) / RB;
   const long long gw = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
   const long long stride = static_cast<long long>(gridDim.x) * WARPS;
   auto src = [&](int k) {
-    return Ptrs{a.outs + k * a.stride_out, a.lses + k * a.stride_lse, false};
+    return Ptrs{a.outs + k * a.stride_out, a.lses + k * a.stride_lse};
   };
   for (long long b = gw; b < nblk; b += stride) {
     const long long row0 = b * RB;
     const int nr = static_cast<int>(min(static_cast<long long>(RB), a.rows - row0));
-    compose_rows<D>(row0, nr, a.n_states, src, a.out, a.lse, lane);
+    compose_rows<D, float>(row0, nr, a.n_states, 0, src, a.out, a.lse, lane);
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(WARPS * 32) compose_plan_kernel(const __grid_constant__ ComposePlan a) {
+// E: type of the cache planes' OUT entries
+template <int D, class E>
+__global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __grid_constant__ ComposePlan a) {
   const int lane = threadIdx.x & 31;
   const int bpp = (a.n + RB - 1) / RB;  // warp blocks per (head, partition)
   const long long nblk = static_cast<long long>(a.B) * a.H * a.P * bpp;
@@ -196,15 +200,22 @@ __global__ void __launch_bounds__(WARPS * 32) compose_plan_kernel(const __grid_c
     const int nr = min(RB, (i + 1) * a.n - s0);
     const long long row0 = bh * a.S + s0;
     const int8_t* list = a.src[i];
+    // branch-free pointer selection: the LSE passes evaluate a different
+    // source in every lane
     auto src = [&](int k) {
       const int j = list[k];
-      if (j == -1) return Ptrs{a.out, a.lse, false};
-      if (j == -2) return Ptrs{a.local_out, a.local_lse, false};
-      if (a.cache_bf16)
-        return Ptrs{static_cast<const __nv_bfloat16*>(a.cache_out) + j * a.plane_out, a.cache_lse + j * a.plane_lse, true};
-      return Ptrs{static_cast<const float*>(a.cache_out) + j * a.plane_out, a.cache_lse + j * a.plane_lse, false};
+      const long long jj = j < 0 ? 0 : j;
+      const void* o = static_cast<const E*>(a.cache_out) + jj * a.plane_out;
+      const float* l = a.cache_lse + jj * a.plane_lse;
+      o = j == -2 ? static_cast<const void*>(a.local_out) : o;
+      l = j == -2 ? a.local_lse : l;
+      o = j == -1 ? static_cast<const void*>(a.out) : o;
+      l = j == -1 ? a.lse : l;
+      return Ptrs{o, l};
     };
-    compose_rows<D>(row0, nr, a.nsrc[i], src, a.out, a.lse, lane);
+    // the fp32 sources (composite, local state) lead the list
+    const int nf = (a.nsrc[i] > 0 && list[0] < 0) + (a.nsrc[i] > 1 && list[1] < 0);
+    compose_rows<D, E>(row0, nr, a.nsrc[i], nf, src, a.out, a.lse, lane);
   }
 }
 
@@ -230,10 +241,14 @@ cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st) {
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st) {
   const long long nblk = static_cast<long long>(a.B) * a.H * a.P * ((a.n + RB - 1) / RB);
   const unsigned grid = static_cast<unsigned>(grid_for(nblk));
-  if (a.d == 128)
-    compose_plan_kernel<128><<<grid, WARPS * 32, 0, st>>>(a);
+  if (a.d == 128 && a.cache_bf16)
+    compose_plan_kernel<128, __nv_bfloat16><<<grid, WARPS * 32, 0, st>>>(a);
+  else if (a.d == 128)
+    compose_plan_kernel<128, float><<<grid, WARPS * 32, 0, st>>>(a);
+  else if (a.d == 64 && a.cache_bf16)
+    compose_plan_kernel<64, __nv_bfloat16><<<grid, WARPS * 32, 0, st>>>(a);
   else if (a.d == 64)
-    compose_plan_kernel<64><<<grid, WARPS * 32, 0, st>>>(a);
+    compose_plan_kernel<64, float><<<grid, WARPS * 32, 0, st>>>(a);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
