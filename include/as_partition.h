@@ -168,7 +168,11 @@ as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step,
  * entry.  h_hit / h_age (may be NULL) as in as_plan_resolve.  The plan is
  * checked before any launch: on AS_ERR_CACHE_MISS or AS_ERR_INVALID_ARG
  * nothing is launched and the cache is unchanged.  The cache must have been
- * initialised for the same B, H, S, d, P. */
+ * initialised for the same B, H, S, d, P.  The call neither allocates nor
+ * synchronises, so it can be captured in a CUDA graph: a replay repeats the
+ * device work with the captured plan and pointers, while the host
+ * bookkeeping (checks, hit/age, t_c, member) happens once, at the captured
+ * call; capture steps that store nothing, or account for that yourself. */
 as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
                   const uint8_t* h_plan, int step, float* out, float* lse,
                   uint8_t* h_hit, int32_t* h_age, void* stream);

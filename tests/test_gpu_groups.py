@@ -226,3 +226,37 @@ def test_cache_checkpoint_and_resume(api, tmp_path):
         torch.cuda.synchronize()
         assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]), t
         assert np.array_equal(a[2], b[2]) and np.array_equal(a[3], b[3])
+
+
+def test_step_replays_from_a_cuda_graph(api):
+    """as_step captured in a CUDA graph (a step whose plan stores nothing, so
+    it has no host bookkeeping): replays give the eager result bit for bit,
+    including after the inputs change in place."""
+    s = W.spec("video_reuse", H=2, rows=8, cols=16, S=16 * 8 * 16)
+    traj = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P)
+    api.as_step(cache, *traj[0], W.plan_for_step(s, 0).numpy(), 0)   # anchor, stores
+    plan = W.plan_for_step(s, 1).numpy()                              # reuse only
+    assert not (plan == W.PLAN_FRESH_STORE).any()
+    q, k, v = (x.clone() for x in traj[1])
+    out = torch.empty((s.B, s.H, s.S, s.d), device="cuda")
+    lse = torch.empty((s.B, s.H, s.S), device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        api.as_step(cache, q, k, v, plan, 1, out=out, lse=lse)       # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        api.as_step(cache, q, k, v, plan, 1, out=out, lse=lse)
+    ref_o, ref_l, _, _ = api.as_step(cache, q, k, v, plan, 1)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    q.copy_(traj[0][0])                                               # new inputs, same buffers
+    ref_o, ref_l, _, _ = api.as_step(cache, q, k, v, plan, 1)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    del graph
