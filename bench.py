@@ -48,6 +48,8 @@ from attention_state_reuse_partition_b200 import workloads as W  # noqa: E402
 
 METRIC = "fresh-partition attn TFLOP/s & compose GB/s at 1 B200; % of bf16/HBM roofline"
 WORKLOAD = "flux_image"
+WORKLOAD_TEXT = (f"{WORKLOAD}: B=1 H=24 S=4608 (4096 image + 512 text) d=128, P=8 partitions of 576, "
+                 "all pairs fresh and composed")
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -566,8 +568,7 @@ def main():
         "metric": METRIC, "value": round(res["value"], 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: B=1 H=24 S=4608 (4096 image + 512 text) d=128, P=8 partitions "
-                               f"of 576, all pairs fresh and composed", "global_batch": world, "seq_len": s.S,
+        "config": {"workload": WORKLOAD_TEXT, "global_batch": world, "seq_len": s.S,
                    "parallelism": f"replicas{world}" if world > 1 else "single", "l2": "flushed (256 MiB write) "
                    "before every timed step"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
@@ -613,8 +614,8 @@ def run_reference(args, rank, world):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{WORKLOAD}: B=1 H=24 S=4608 d=128, P=8, all pairs fresh (3 heads per step)",
-                   "global_batch": 1, "seq_len": s.S, "parallelism": "host cores"},
+        "config": {"workload": WORKLOAD_TEXT, "global_batch": 1, "seq_len": s.S,
+                   "parallelism": "host cores (float64 oracle)"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
