@@ -90,39 +90,57 @@ struct Ptrs {
 // others in E (fp32 or bf16), so that every batch of loads has one type.  The
 // output may alias a source: every source row is read before the output row
 // is written, by the same warp.
-template <int D, class E, class SrcFn>
+template <int D, class E, int UNROLL, class SrcFn>
 __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, int nf, SrcFn src, float* out,
                                              float* lse, int lane) {
   using V = Vec<D>;
   using T = typename V::T;
-  float m[RB], tot[RB];
+  float m[RB], tot[RB], inv[RB];
+  // up to 32 sources (one per lane; the common case): lane k loads the LSEs
+  // of source k once and keeps them, and each weight is one exponential
+  float ev[RB];
+  const bool one_chunk = nsrc <= 32;
+  if (one_chunk) {
+    const float* lb = lane < nsrc ? src(lane).second + row0 : nullptr;
 #pragma unroll
-  for (int rr = 0; rr < RB; ++rr) m[rr] = -INFINITY;
-  for (int k0 = 0; k0 < nsrc; k0 += 32) {
-    const int k = k0 + lane;
-    if (k < nsrc) {
-      const float* lb = src(k).second + row0;
+    for (int rr = 0; rr < RB; ++rr) ev[rr] = (lb != nullptr && rr < nr) ? lb[rr] : -INFINITY;
 #pragma unroll
-      for (int rr = 0; rr < RB; ++rr)
-        if (rr < nr) m[rr] = fmaxf(m[rr], lb[rr]);
+    for (int rr = 0; rr < RB; ++rr) m[rr] = warp_max(ev[rr]);
+#pragma unroll
+    for (int rr = 0; rr < RB; ++rr) ev[rr] = m[rr] != -INFINITY ? __expf(ev[rr] - m[rr]) : 0.f;
+#pragma unroll
+    for (int rr = 0; rr < RB; ++rr) tot[rr] = warp_sum(ev[rr]);
+  } else {
+#pragma unroll
+    for (int rr = 0; rr < RB; ++rr) m[rr] = -INFINITY;
+    for (int k0 = 0; k0 < nsrc; k0 += 32) {
+      const int k = k0 + lane;
+      if (k < nsrc) {
+        const float* lb = src(k).second + row0;
+#pragma unroll
+        for (int rr = 0; rr < RB; ++rr)
+          if (rr < nr) m[rr] = fmaxf(m[rr], lb[rr]);
+      }
     }
-  }
 #pragma unroll
-  for (int rr = 0; rr < RB; ++rr) {
-    m[rr] = warp_max(m[rr]);
-    tot[rr] = 0.f;
-  }
-  for (int k0 = 0; k0 < nsrc; k0 += 32) {
-    const int k = k0 + lane;
-    if (k < nsrc) {
-      const float* lb = src(k).second + row0;
-#pragma unroll
-      for (int rr = 0; rr < RB; ++rr)
-        if (rr < nr && m[rr] != -INFINITY) tot[rr] += expf(lb[rr] - m[rr]);
+    for (int rr = 0; rr < RB; ++rr) {
+      m[rr] = warp_max(m[rr]);
+      tot[rr] = 0.f;
     }
+    for (int k0 = 0; k0 < nsrc; k0 += 32) {
+      const int k = k0 + lane;
+      if (k < nsrc) {
+        const float* lb = src(k).second + row0;
+#pragma unroll
+        for (int rr = 0; rr < RB; ++rr)
+          if (rr < nr && m[rr] != -INFINITY) tot[rr] += __expf(lb[rr] - m[rr]);
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < RB; ++rr) tot[rr] = warp_sum(tot[rr]);
   }
 #pragma unroll
-  for (int rr = 0; rr < RB; ++rr) tot[rr] = warp_sum(tot[rr]);
+  for (int rr = 0; rr < RB; ++rr) inv[rr] = tot[rr] > 0.f ? 1.0f / tot[rr] : 0.f;
 
   T acc[RB];
 #pragma unroll
@@ -130,11 +148,14 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, i
   for (int k0 = 0; k0 < nsrc; k0 += 32) {
     const int k = k0 + lane;
     float coef[RB];
-    if (k < nsrc) {
+    if (one_chunk) {
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr) coef[rr] = ev[rr] * inv[rr];
+    } else if (k < nsrc) {
       const float* lb = src(k).second + row0;
 #pragma unroll
       for (int rr = 0; rr < RB; ++rr)
-        coef[rr] = (rr < nr && tot[rr] > 0.f) ? expf(lb[rr] - m[rr]) / tot[rr] : 0.f;
+        coef[rr] = (rr < nr && tot[rr] > 0.f) ? __expf(lb[rr] - m[rr]) * inv[rr] : 0.f;
     } else {
 #pragma unroll
       for (int rr = 0; rr < RB; ++rr) coef[rr] = 0.f;
@@ -142,6 +163,7 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, i
     const int kn = min(32, nsrc - k0);
     // one source at a time (its pointers resolved once), its rows' loads in
     // flight together
+#pragma unroll UNROLL
     for (int kk = 0; kk < kn; ++kk) {
       const Ptrs sp = src(k0 + kk);
       T x[RB];
@@ -163,7 +185,7 @@ __device__ __forceinline__ void compose_rows(long long row0, int nr, int nsrc, i
   for (int rr = 0; rr < RB; ++rr) {
     if (rr >= nr) break;
     reinterpret_cast<T*>(out + (row0 + rr) * D)[lane] = acc[rr];
-    if (lane == 0) lse[row0 + rr] = tot[rr] > 0.f ? m[rr] + logf(tot[rr]) : -INFINITY;
+    if (lane == 0) lse[row0 + rr] = tot[rr] > 0.f ? m[rr] + __logf(tot[rr]) : -INFINITY;
   }
 }
 
@@ -179,7 +201,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_strided_kernel(const __
   for (long long b = gw; b < nblk; b += stride) {
     const long long row0 = b * RB;
     const int nr = static_cast<int>(min(static_cast<long long>(RB), a.rows - row0));
-    compose_rows<D, float>(row0, nr, a.n_states, 0, src, a.out, a.lse, lane);
+    compose_rows<D, float, 2>(row0, nr, a.n_states, 0, src, a.out, a.lse, lane);
   }
 }
 
@@ -200,7 +222,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
     const int nr = min(RB, (i + 1) * a.n - s0);
     const long long row0 = bh * a.S + s0;
     const int8_t* list = a.src[i];
-    // branch-free pointer selection: the LSE passes evaluate a different
+    // branch-free pointer selection: the LSE pass evaluates a different
     // source in every lane
     auto src = [&](int k) {
       const int j = list[k];
@@ -215,7 +237,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
     };
     // the fp32 sources (composite, local state) lead the list
     const int nf = (a.nsrc[i] > 0 && list[0] < 0) + (a.nsrc[i] > 1 && list[1] < 0);
-    compose_rows<D, E>(row0, nr, a.nsrc[i], nf, src, a.out, a.lse, lane);
+    // measured: bf16 planes (half the bytes per load) gain from two sources'
+    // loads in flight, fp32 planes do not
+    compose_rows<D, E, sizeof(E) == 2 ? 2 : 1>(row0, nr, a.nsrc[i], nf, src, a.out, a.lse, lane);
   }
 }
 
