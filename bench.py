@@ -369,12 +369,16 @@ def run_compose(args, device):
 
 
 def run_reuse(args, device):
-    """Two-step video reuse: anchor step then a reuse step (window 2)."""
+    """Two-step video reuse: anchor step then a reuse step (window 2).
+    ``--reuse-heads`` runs fewer heads (a smaller case for profiling);
+    ``--reuse-groups`` / ``--reuse-cache`` set the cache's group size and
+    entry type."""
     from attention_state_reuse_partition_b200 import api
-    s = W.spec("video_reuse")
+    s = W.spec("video_reuse") if args.reuse_heads is None else W.spec("video_reuse", H=args.reuse_heads)
+    g, cdt = args.reuse_groups, args.reuse_cache
     steps = [(q, k, v) for _, q, k, v in W.video_trajectory(s, device=device)]
-    plans = [W.plan_for_step(s, t).numpy() for t in range(s.steps)]
-    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    plans = [W.grouped_plan_for_step(s, t, g).numpy() for t in range(s.steps)]
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, g=g, cache_dtype=cdt)
     out = torch.empty((s.B, s.H, s.S, s.d), device=device)
     lse = torch.empty((s.B, s.H, s.S), device=device)
     q1, k1, v1 = steps[1]
@@ -383,7 +387,7 @@ def run_reuse(args, device):
     fresh_flops = 4.0 * s.B * s.H * n_fresh * s.n * s.n * s.d
     times = []
     for rep in range(4):
-        c = api.AsCache(s.B, s.H, s.S, s.d, s.P, buffer=cache.buffer)
+        c = api.AsCache(s.B, s.H, s.S, s.d, s.P, buffer=cache.buffer, g=g, cache_dtype=cdt)
         api.as_step(c, *steps[0], plans[0], 0, out=out, lse=lse)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -397,11 +401,16 @@ def run_reuse(args, device):
     full_o, _ = api.as_partition_attn(q1, k1, v1, s.P, -1, list(range(s.P)))
     torch.cuda.synchronize()
     mse = torch.mean((out - full_o) ** 2).item()
-    state_bytes = s.B * s.H * s.n * (s.d + 1) * 4
-    reuse_bytes = n_reuse * state_bytes
+    entry_bytes = s.B * s.H * s.n * (s.d * (2 if cdt == "bf16" else 4) + 4)  # one (i, G) entry
+    NG = (s.P + g - 1) // g
+    reused_entries = sum(bool((plans[1][i, G * g:(G + 1) * g] == W.PLAN_REUSE).any())
+                         for i in range(s.P) for G in range(NG))
+    reuse_bytes = reused_entries * entry_bytes
     del cache, steps, full_o
     torch.cuda.empty_cache()
-    return {"workload": "video_reuse step t", "ms": ms, "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
+    name = "video_reuse step t" + ("" if (g, cdt, s.H) == (1, "f32", 24) else f" (H={s.H}, g={g}, {cdt} entries)")
+    return {"workload": name, "ms": ms, "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
+            "reused_entries": reused_entries,
             "fresh_tflops_whole_step": fresh_flops / (ms * 1e-3) / 1e12, "reuse_bytes": reuse_bytes,
             "reuse_mse_vs_full": mse}
 
@@ -513,6 +522,9 @@ def main():
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
+    ap.add_argument("--reuse-heads", type=int, default=None, help="heads of the reuse workload (default 24)")
+    ap.add_argument("--reuse-groups", type=int, default=1, help="cache group size of the reuse workload")
+    ap.add_argument("--reuse-cache", choices=["f32", "bf16"], default="f32", help="cache entry type of the reuse workload")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device-resident step only (no e2e, CPU baseline or secondary workloads)")
     args = ap.parse_args()
