@@ -121,13 +121,14 @@ def weak_scaling_value(units_per_rank: float, world: int, ms_max: float) -> floa
 
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons through NVML (read-only
-    queries) every 10 ms in a background thread.  Samples taken inside the
-    timed region are marked via ``mark_timed``."""
+    queries) every 2 ms in a background thread, so that even a timed region of
+    a few milliseconds holds samples.  Samples taken inside the timed region
+    are marked via ``mark_timed``."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int, interval: float = 0.01):
+    def __init__(self, gpu_index: int, interval: float = 0.002):
         import threading
         self.gpu, self.interval = gpu_index, interval
         self.samples = []
@@ -175,7 +176,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": float(use[0][2]),
                 "reasons": reasons, "samples_timed": len(timed), "samples_total": len(self.samples),
                 "power_w_max": max(x[3] for x in use),
-                "how": "NVML every 10 ms; median over the samples inside the timed region "
+                "how": "NVML every 2 ms; median over the samples inside the timed region "
                        "(all samples, warm-up included, when the region is shorter than one interval)"}
 
 
@@ -511,7 +512,7 @@ def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cac
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
     ap.add_argument("--no-secondary", action="store_true")
