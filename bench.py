@@ -422,7 +422,8 @@ def run_video_long(args, device, g=1, cache_dtype="f32"):
     g > 1 the cache keeps one composed entry per (query partition, group of g
     KV partitions) and a forced pair refreshes its whole group."""
     from attention_state_reuse_partition_b200 import api
-    s = W.spec("video_long")
+    heads = getattr(args, "video_heads", None)
+    s = W.spec("video_long") if heads is None else W.spec("video_long", H=heads)
     cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, g=g, cache_dtype=cache_dtype)
     NG = (s.P + g - 1) // g
     entry_bytes = s.B * s.H * s.n * (s.d * (2 if cache_dtype == "bf16" else 4) + 4)  # one (i, G) entry
@@ -458,6 +459,8 @@ def run_video_long(args, device, g=1, cache_dtype="f32"):
     torch.cuda.empty_cache()
     name = "video_long (4 steps)" if g == 1 and cache_dtype == "f32" else \
         f"video_long (4 steps), cache groups of {g} partitions, {cache_dtype} OUT entries"
+    if heads is not None:
+        name += f" with {s.H} heads"
     return {"workload": name, "g": g, "cache_dtype": cache_dtype, "cache_gb": round(cache_gb, 2),
             "steps": per_step, "reuse_mse_vs_full_last_step": mse}
 
@@ -469,7 +472,8 @@ def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cac
     statistics after anchor steps.  With g > 1 the planner decides per cache
     group of g KV partitions."""
     from attention_state_reuse_partition_b200 import api
-    s = W.spec("video_long")
+    heads = getattr(args, "video_heads", None)
+    s = W.spec("video_long") if heads is None else W.spec("video_long", H=heads)
     cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, g=g, cache_dtype=cache_dtype)
     pl = api.AsPlanner(s.P, window, reuse_ratio, eps_local, s.B, s.H, s.S, s.d, device=device, g=g)
     out = torch.empty((s.B, s.H, s.S, s.d), device=device)
@@ -524,6 +528,8 @@ def main():
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
     ap.add_argument("--reuse-heads", type=int, default=None, help="heads of the reuse workload (default 24)")
+    ap.add_argument("--video-heads", type=int, default=None,
+                    help="heads of the video_long workloads (default 40; fewer for a small profiling case)")
     ap.add_argument("--reuse-groups", type=int, default=1, help="cache group size of the reuse workload")
     ap.add_argument("--reuse-cache", choices=["f32", "bf16"], default="f32", help="cache entry type of the reuse workload")
     ap.add_argument("--kernel-only", action="store_true",
