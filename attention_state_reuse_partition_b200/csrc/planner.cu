@@ -87,15 +87,31 @@ __global__ void __launch_bounds__(THREADS) stats_partials_kernel(const OutT* __r
   const float* lse_ij = cache_lse + j * plane_lse + row0;
   const float* lse_i = lse_full + row0;
   const OutT* out_ij = cache_out + j * plane_out + row0 * d;
-  double ws = 0.0, sq = 0.0;
+  double ws = 0.0;
   for (int r = threadIdx.x; r < n; r += THREADS) ws += exp(static_cast<double>(lse_ij[r]) - lse_i[r]);
-  const long long count = static_cast<long long>(n) * d;
-  for (long long e = threadIdx.x; e < count; e += THREADS) {
-    const double o = static_cast<float>(out_ij[e]);
-    sq += o * o;
+  // the entry's n rows of OUT are contiguous: 16-byte loads, every element
+  // squared and summed in fp64 over four independent accumulators
+  constexpr int EPV = 16 / static_cast<int>(sizeof(OutT));  // elements per 16-byte vector
+  const long long nvec = static_cast<long long>(n) * d / EPV;
+  const uint4* vec = reinterpret_cast<const uint4*>(out_ij);
+  double sq4[4] = {0.0, 0.0, 0.0, 0.0};
+  for (long long e = threadIdx.x; e < nvec; e += THREADS) {
+    const uint4 u = vec[e];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if constexpr (sizeof(OutT) == 2) {
+        const double lo = __uint_as_float(w[c] << 16), hi = __uint_as_float(w[c] & 0xffff0000u);
+        sq4[c] = fma(lo, lo, sq4[c]);
+        sq4[c] = fma(hi, hi, sq4[c]);
+      } else {
+        const double x = __uint_as_float(w[c]);
+        sq4[c] = fma(x, x, sq4[c]);
+      }
+    }
   }
   const double sws = block_sum(ws, sh);
-  const double ssq = block_sum(sq, sh);
+  const double ssq = block_sum((sq4[0] + sq4[1]) + (sq4[2] + sq4[3]), sh);
   if (threadIdx.x == 0) {
     partials[(static_cast<long long>(pair) * BH + bh) * 2 + 0] = sws;
     partials[(static_cast<long long>(pair) * BH + bh) * 2 + 1] = ssq;
