@@ -47,16 +47,25 @@ __global__ void __launch_bounds__(THREADS) drift_partials_kernel(const float* __
   __shared__ double sh[THREADS / 32];
   const int i = blockIdx.x, bh = blockIdx.y;
   const long long base = (static_cast<long long>(bh) * S + static_cast<long long>(i) * n) * d;
-  const long long count = static_cast<long long>(n) * d;
-  double dd = 0.0, aa = 0.0;
-  for (long long e = threadIdx.x; e < count; e += THREADS) {
-    const double a = anchor[base + e];
-    const double x = now[base + e] - a;
-    dd += x * x;
-    aa += a * a;
+  // the partition's n rows are contiguous: 16-byte loads, each element's
+  // difference and square in fp64, four independent accumulators per sum
+  const long long nvec = static_cast<long long>(n) * d / 4;
+  const float4* nv = reinterpret_cast<const float4*>(now + base);
+  const float4* av = reinterpret_cast<const float4*>(anchor + base);
+  double dd[4] = {0.0, 0.0, 0.0, 0.0}, aa[4] = {0.0, 0.0, 0.0, 0.0};
+  for (long long e = threadIdx.x; e < nvec; e += THREADS) {
+    const float4 x4 = nv[e], a4 = av[e];
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w}, as[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const double a = as[c];
+      const double x = static_cast<double>(xs[c]) - a;
+      dd[c] = fma(x, x, dd[c]);
+      aa[c] = fma(a, a, aa[c]);
+    }
   }
-  const double sdd = block_sum(dd, sh);
-  const double saa = block_sum(aa, sh);
+  const double sdd = block_sum((dd[0] + dd[1]) + (dd[2] + dd[3]), sh);
+  const double saa = block_sum((aa[0] + aa[1]) + (aa[2] + aa[3]), sh);
   if (threadIdx.x == 0) {
     partials[(static_cast<long long>(i) * BH + bh) * 2 + 0] = sdd;
     partials[(static_cast<long long>(i) * BH + bh) * 2 + 1] = saa;
