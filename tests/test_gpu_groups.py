@@ -260,3 +260,23 @@ def test_step_replays_from_a_cuda_graph(api):
     torch.cuda.synchronize()
     assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
     del graph
+
+
+@pytest.mark.parametrize("P,n,d", [(1, 640, 128), (8, 8, 64), (16, 8, 128)])
+def test_step_extreme_partitions(api, P, n, d):
+    """One partition (the first step is plain attention, stored; the next
+    ones take the whole row from the cache), and partitions of 8 tokens
+    (every KV range and query block far shorter than a 128-row tile): the
+    same bookkeeping and states as the oracle over three steps."""
+    s = W.spec("flux_image", B=1, H=2, S=P * n, d=d, P=P)
+    q, k, v = (x.cuda() for x in W.flux_qkv(s))
+    gen = torch.Generator(device="cuda").manual_seed(70 + P)
+    steps = [(q, (k.float() + 0.05 * t * torch.randn(k.shape, generator=gen, device="cuda")).to(k.dtype), v)
+             for t in range(3)]
+    near = np.abs(np.arange(P)[:, None] - np.arange(P)[None, :]) <= 1
+    anchor = np.where(near, W.PLAN_FRESH, W.PLAN_FRESH_STORE).astype(np.uint8)
+    reuse = np.where(near, W.PLAN_FRESH, W.PLAN_REUSE).astype(np.uint8)
+    if P == 1:
+        anchor[:] = W.PLAN_FRESH_STORE
+        reuse[:] = W.PLAN_REUSE
+    _run_grouped(api, s, steps, [anchor, reuse, reuse], 1, "f32")
