@@ -280,3 +280,23 @@ def test_step_extreme_partitions(api, P, n, d):
         anchor[:] = W.PLAN_FRESH_STORE
         reuse[:] = W.PLAN_REUSE
     _run_grouped(api, s, steps, [anchor, reuse, reuse], 1, "f32")
+
+
+@pytest.mark.parametrize("cache_dt", ["f32", "bf16"])
+def test_step_many_sources(api, cache_dt):
+    """Rows with more than 32 sources, so the step compose takes its general
+    path: 40 partitions, every pair stored at the first step and reused at
+    the next ones (40 cache entries per row), plus a row mixing fresh, stored
+    and reused pairs."""
+    P, n = 40, 16
+    s = W.spec("flux_image", B=1, H=2, S=P * n, d=64, P=P)
+    q, k, v = (x.cuda() for x in W.flux_qkv(s))
+    gen = torch.Generator(device="cuda").manual_seed(91)
+    steps = [(q, (k.float() + 0.05 * t * torch.randn(k.shape, generator=gen, device="cuda")).to(k.dtype), v)
+             for t in range(3)]
+    stored = np.full((P, P), W.PLAN_FRESH_STORE, np.uint8)
+    reuse = np.zeros((P, P), np.uint8)
+    mixed = reuse.copy()
+    mixed[5, :10] = W.PLAN_FRESH
+    mixed[5, 10:20] = W.PLAN_FRESH_STORE
+    _run_grouped(api, s, steps, [stored, reuse, mixed], 1, cache_dt)
