@@ -115,6 +115,37 @@ def test_attn_f32_tiny(api):
         check_f32(oi, li, ref_o, ref_l, f"f32 q_part {i}")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_attn_and_step_with_a_given_scale(api, dtype):
+    """A softmax scale other than 1/sqrt(d), through the CUDA-core (fp32) and
+    the tensor-core (bf16) kernels and through a reuse step."""
+    scale = 0.2
+    if dtype == "f32":
+        s = W.spec("tiny_f32")
+        q, k, v = W.iid_qkv(s)
+        check = check_f32
+    else:
+        s = W.spec("flux_image", H=2, S=640, P=5)
+        q, k, v = W.flux_qkv(s)
+        check = check_bf16
+    qn, kn, vn = (x.double().numpy() for x in (q, k, v))
+    qc, kc, vc = (x.cuda() for x in (q, k, v))
+    full_o, full_l = O.full_attention(qn, kn, vn, scale)
+    out, lse = api.as_partition_attn(qc, kc, vc, s.P, -1, list(range(s.P)), scale=scale)
+    check(out, lse, full_o, full_l, f"{dtype} attention, scale {scale}")
+    P = s.P
+    near = np.abs(np.arange(P)[:, None] - np.arange(P)[None, :]) <= 1
+    anchor_plan = np.where(near, 1, 2).astype(np.uint8)
+    reuse_plan = np.where(near, 1, 0).astype(np.uint8)
+    cache = api.AsCache(s.B, s.H, s.S, s.d, P)
+    ocache = O.StateCache(P)
+    for t, plan in enumerate([anchor_plan, reuse_plan]):
+        out, lse, hit, age = api.as_step(cache, qc, kc, vc, plan, t, scale=scale)
+        ref_o, ref_l, ref_hit, ref_age = O.step(ocache, qn, kn, vn, plan, t, scale)
+        assert np.array_equal(hit, ref_hit) and np.array_equal(age, ref_age)
+        check(out, lse, ref_o, ref_l, f"{dtype} step {t}, scale {scale}")
+
+
 # ---------------------------------------------------------------------------
 # bf16 partition attention (tensor cores)
 # ---------------------------------------------------------------------------
