@@ -29,6 +29,18 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise AsError(_lib.AS_ERR_INVALID_ARG, f"unsupported input dtype {t.dtype}")
 
 
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
+    """Q, K and V must agree in shape [B, H, S, d], dtype and device: the
+    library reads all three with Q's element type."""
+    if q.dim() != 4:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, f"q must be [B, H, S, d], got shape {tuple(q.shape)}")
+    for name, t in (("k", k), ("v", v)):
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise AsError(_lib.AS_ERR_INVALID_ARG,
+                          f"{name} ({tuple(t.shape)}, {t.dtype}, {t.device}) does not match q "
+                          f"({tuple(q.shape)}, {q.dtype}, {q.device})")
+
+
 def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream or None
@@ -48,6 +60,7 @@ def as_partition_attn(q, k, v, P: int, q_part: int, kv_parts: Sequence[int], com
                       scale: Optional[float] = None, out=None, lse=None, stream=None):
     """States of query partition ``q_part`` (or all rows, q_part=-1) against
     the listed KV partitions; composed (compose=True) or one per partition."""
+    _check_qkv(q, k, v)
     B, H, S, d = q.shape
     R = S if q_part < 0 else S // P
     scale = 1.0 / d ** 0.5 if scale is None else scale
@@ -206,6 +219,7 @@ def as_plan_resolve(cache: AsCache, plan, step: int):
 def as_step(cache: AsCache, q, k, v, plan, step: int, scale: Optional[float] = None, out=None, lse=None,
             stream=None):
     """One step under a compute/reuse plan; returns (out, lse, hit, age)."""
+    _check_qkv(q, k, v)
     B, H, S, d = q.shape
     P = cache.P
     scale = 1.0 / d ** 0.5 if scale is None else scale
@@ -227,6 +241,7 @@ def as_step_local(cache: AsCache, q, k, v, plan, step: int, local_out, local_lse
     """as_step with the step's local states AS(i, i) given (from
     as_local_states on the same inputs): plain-fresh diagonal pairs are
     composed from them instead of recomputed.  Returns (out, lse, hit, age)."""
+    _check_qkv(q, k, v)
     B, H, S, d = q.shape
     P = cache.P
     scale = 1.0 / d ** 0.5 if scale is None else scale
@@ -302,6 +317,7 @@ def as_planner_init(P, window, reuse_ratio, eps_local, B=0, H=0, S=0, d=0, devic
 
 def as_local_states(q, k, v, P: int, scale: Optional[float] = None, out=None, lse=None, stream=None):
     """Local states AS(i, i) of every query partition: out [B,H,S,d], lse [B,H,S]."""
+    _check_qkv(q, k, v)
     B, H, S, d = q.shape
     scale = 1.0 / d ** 0.5 if scale is None else scale
     if out is None:

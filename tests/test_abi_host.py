@@ -298,3 +298,23 @@ def test_cache_bookkeeping_round_trip(api):
     other.set_t_c(sd["t_c"])
     other.set_member(sd["member"])
     assert np.array_equal(other.t_c, t_c) and np.array_equal(other.member, member)
+
+
+def test_python_entry_points_check_q_k_v(api):
+    """The binding refuses K or V that differ from Q in shape or dtype (the
+    library would read them with Q's element type), before any device call."""
+    import torch
+    from attention_state_reuse_partition_b200 import _lib
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    good = torch.zeros_like(q)
+    cache = api.AsCache.host_only(1, 2, 64, 64, 4)
+    plan = np.ones((4, 4), np.uint8)
+    calls = [lambda k, v: api.as_partition_attn(q, k, v, 4, -1, [0, 1, 2, 3]),
+             lambda k, v: api.as_step(cache, q, k, v, plan, 0),
+             lambda k, v: api.as_local_states(q, k, v, 4)]
+    for bad, what in [(good.float(), "dtype"), (torch.zeros(1, 2, 32, 64, dtype=torch.bfloat16), "shape")]:
+        for fn in calls:
+            for args in [(bad, good), (good, bad)]:
+                with pytest.raises(api.AsError) as ei:
+                    fn(*args)
+                assert ei.value.status == _lib.AS_ERR_INVALID_ARG and "does not match q" in str(ei.value), what
