@@ -41,6 +41,18 @@ def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
                           f"({tuple(q.shape)}, {q.dtype}, {q.device})")
 
 
+def _buf(t: Optional[torch.Tensor], shape, device, name: str) -> torch.Tensor:
+    """An fp32 buffer of exactly `shape`: allocated when not given, checked
+    when given (the library writes all of it)."""
+    shape = tuple(int(x) for x in shape)
+    if t is None:
+        return torch.empty(shape, device=device, dtype=torch.float32)
+    if t.dtype != torch.float32 or tuple(t.shape) != shape:
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"{name} must be float32 of shape {shape}, got {t.dtype} of shape {tuple(t.shape)}")
+    return t
+
+
 def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream or None
@@ -65,10 +77,8 @@ def as_partition_attn(q, k, v, P: int, q_part: int, kv_parts: Sequence[int], com
     R = S if q_part < 0 else S // P
     scale = 1.0 / d ** 0.5 if scale is None else scale
     planes = () if compose else (len(kv_parts),)
-    if out is None:
-        out = torch.empty(planes + (B, H, R, d), device=q.device, dtype=torch.float32)
-    if lse is None:
-        lse = torch.empty(planes + (B, H, R), device=q.device, dtype=torch.float32)
+    out = _buf(out, planes + (B, H, R, d), q.device, "out")
+    lse = _buf(lse, planes + (B, H, R), q.device, "lse")
     parts = (ctypes.c_int32 * len(kv_parts))(*[int(x) for x in kv_parts])
     check(LIB.as_partition_attn(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q), B, H, S, d, P,
                                 float(scale), int(q_part), parts, len(kv_parts), 1 if compose else 0,
@@ -80,11 +90,13 @@ def as_compose(outs, lses, out=None, lse=None, stream=None):
     """Compose N states per row: outs [N, ..., d], lses [N, ...] (fp32)."""
     N = outs.shape[0]
     d = outs.shape[-1]
+    if outs.dtype != torch.float32 or lses.dtype != torch.float32 or tuple(lses.shape) != tuple(outs.shape[:-1]):
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"outs [N, ..., d] and lses [N, ...] must be float32 with matching shapes, got "
+                      f"{outs.dtype} {tuple(outs.shape)} and {lses.dtype} {tuple(lses.shape)}")
     rows = lses[0].numel()
-    if out is None:
-        out = torch.empty(outs.shape[1:], device=outs.device, dtype=torch.float32)
-    if lse is None:
-        lse = torch.empty(lses.shape[1:], device=lses.device, dtype=torch.float32)
+    out = _buf(out, outs.shape[1:], outs.device, "out")
+    lse = _buf(lse, lses.shape[1:], lses.device, "lse")
     check(LIB.as_compose(_dev(outs, "outs"), _dev(lses, "lses"), N, rows, d, rows * d, rows,
                          _dev(out, "out"), _dev(lse, "lse"), _stream_ptr(stream)))
     return out, lse
@@ -223,10 +235,8 @@ def as_step(cache: AsCache, q, k, v, plan, step: int, scale: Optional[float] = N
     B, H, S, d = q.shape
     P = cache.P
     scale = 1.0 / d ** 0.5 if scale is None else scale
-    if out is None:
-        out = torch.empty((B, H, S, d), device=q.device, dtype=torch.float32)
-    if lse is None:
-        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    out = _buf(out, (B, H, S, d), q.device, "out")
+    lse = _buf(lse, (B, H, S), q.device, "lse")
     arr = _plan_bytes(plan, P)
     hit = np.zeros(P * P, dtype=np.uint8)
     age = np.zeros(P * P, dtype=np.int32)
@@ -245,10 +255,10 @@ def as_step_local(cache: AsCache, q, k, v, plan, step: int, local_out, local_lse
     B, H, S, d = q.shape
     P = cache.P
     scale = 1.0 / d ** 0.5 if scale is None else scale
-    if out is None:
-        out = torch.empty((B, H, S, d), device=q.device, dtype=torch.float32)
-    if lse is None:
-        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    out = _buf(out, (B, H, S, d), q.device, "out")
+    lse = _buf(lse, (B, H, S), q.device, "lse")
+    _buf(local_out, (B, H, S, d), q.device, "local_out")
+    _buf(local_lse, (B, H, S), q.device, "local_lse")
     arr = _plan_bytes(plan, P)
     hit = np.zeros(P * P, dtype=np.uint8)
     age = np.zeros(P * P, dtype=np.int32)
@@ -320,17 +330,23 @@ def as_local_states(q, k, v, P: int, scale: Optional[float] = None, out=None, ls
     _check_qkv(q, k, v)
     B, H, S, d = q.shape
     scale = 1.0 / d ** 0.5 if scale is None else scale
-    if out is None:
-        out = torch.empty((B, H, S, d), device=q.device, dtype=torch.float32)
-    if lse is None:
-        lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32)
+    out = _buf(out, (B, H, S, d), q.device, "out")
+    lse = _buf(lse, (B, H, S), q.device, "lse")
     check(LIB.as_local_states(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dtype_code(q), B, H, S, d, P,
                               float(scale), _dev(out, "out"), _dev(lse, "lse"), _stream_ptr(stream)))
     return out, lse
 
 
+def _check_drift_inputs(now, anchor):
+    if now.dim() != 4 or now.dtype != torch.float32 or anchor.dtype != torch.float32 or anchor.shape != now.shape:
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"now and anchor must be float32 [B, H, S, d] of one shape, got {now.dtype} "
+                      f"{tuple(now.shape)} and {anchor.dtype} {tuple(anchor.shape)}")
+
+
 def as_plan_drift(now, anchor, P: int, scratch, stream=None):
     """(drift [P], norm [P]) of every partition's local state against the anchor's."""
+    _check_drift_inputs(now, anchor)
     B, H, S, d = now.shape
     drift = np.zeros(P, dtype=np.float64)
     norm = np.zeros(P, dtype=np.float64)
@@ -344,6 +360,7 @@ def as_plan_drift_static(now, anchor, P: int, stream=None):
     """as_plan_drift with the library's fixed scratch: for callers that cannot
     allocate device memory (see include/as_partition.h).  The library
     allocates nothing; the limit is P * (B*H*2 + 2) <= 131072."""
+    _check_drift_inputs(now, anchor)
     B, H, S, d = now.shape
     drift = np.zeros(P, dtype=np.float64)
     norm = np.zeros(P, dtype=np.float64)

@@ -318,3 +318,31 @@ def test_python_entry_points_check_q_k_v(api):
                 with pytest.raises(api.AsError) as ei:
                     fn(*args)
                 assert ei.value.status == _lib.AS_ERR_INVALID_ARG and "does not match q" in str(ei.value), what
+
+
+def test_python_entry_points_check_buffers(api):
+    """Caller-supplied outputs must be fp32 of exactly the shape the library
+    writes; compose and drift inputs must agree with each other."""
+    import torch
+    from attention_state_reuse_partition_b200 import _lib
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    cache = api.AsCache.host_only(1, 2, 64, 64, 4)
+    plan = np.ones((4, 4), np.uint8)
+    short = torch.zeros(1, 2, 32, 64)
+    bad_cases = [
+        lambda: api.as_step(cache, q, q, q, plan, 0, out=short),
+        lambda: api.as_step(cache, q, q, q, plan, 0, lse=torch.zeros(1, 2, 64, dtype=torch.float64)),
+        lambda: api.as_partition_attn(q, q, q, 4, 1, [0, 1], out=torch.zeros(1, 2, 64, 64)),
+        lambda: api.as_partition_attn(q, q, q, 4, -1, [0, 1], compose=False, lse=torch.zeros(1, 2, 64)),
+        lambda: api.as_local_states(q, q, q, 4, out=short),
+        lambda: api.as_step_local(cache, q, q, q, plan, 0, short, torch.zeros(1, 2, 64)),
+        lambda: api.as_compose(torch.zeros(3, 10, 64), torch.zeros(3, 11)),
+        lambda: api.as_compose(torch.zeros(3, 10, 64), torch.zeros(3, 10), out=torch.zeros(10, 32)),
+        lambda: api.as_plan_drift(torch.zeros(1, 2, 64, 64), torch.zeros(1, 2, 64, 32), 4, torch.zeros(8)),
+        lambda: api.as_plan_drift_static(torch.zeros(1, 2, 64, 64), torch.zeros(1, 2, 64, 64).double(), 4),
+    ]
+    for k, fn in enumerate(bad_cases):
+        with pytest.raises(api.AsError) as ei:
+            fn()
+        assert ei.value.status == _lib.AS_ERR_INVALID_ARG, (k, str(ei.value))
+        assert "float32" in str(ei.value), (k, str(ei.value))  # not the later device-pointer check
