@@ -232,6 +232,7 @@ def as_step(cache: AsCache, q, k, v, plan, step: int, scale: Optional[float] = N
             stream=None):
     """One step under a compute/reuse plan; returns (out, lse, hit, age)."""
     _check_qkv(q, k, v)
+    _check_cache_shape(cache, q)
     B, H, S, d = q.shape
     P = cache.P
     scale = 1.0 / d ** 0.5 if scale is None else scale
@@ -252,6 +253,7 @@ def as_step_local(cache: AsCache, q, k, v, plan, step: int, local_out, local_lse
     as_local_states on the same inputs): plain-fresh diagonal pairs are
     composed from them instead of recomputed.  Returns (out, lse, hit, age)."""
     _check_qkv(q, k, v)
+    _check_cache_shape(cache, q)
     B, H, S, d = q.shape
     P = cache.P
     scale = 1.0 / d ** 0.5 if scale is None else scale
@@ -337,6 +339,14 @@ def as_local_states(q, k, v, P: int, scale: Optional[float] = None, out=None, ls
     return out, lse
 
 
+def _check_cache_shape(cache: "AsCache", q: torch.Tensor) -> None:
+    """The step reads Q, K, V and writes OUT with the cache's B, H, S, d."""
+    want = (cache.B, cache.H, cache.S, cache.d)
+    if tuple(q.shape) != want:
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"q, k, v must have the cache's shape {want} (B, H, S, d), got {tuple(q.shape)}")
+
+
 def _check_drift_inputs(now, anchor):
     if now.dim() != 4 or now.dtype != torch.float32 or anchor.dtype != torch.float32 or anchor.shape != now.shape:
         raise AsError(_lib.AS_ERR_INVALID_ARG,
@@ -381,8 +391,18 @@ def as_plan_select(ase, window: int, reuse_ratio: float, g: int = 1):
     return plan.reshape(P, P)
 
 
+def _check_planner_state(pl: AsPlanner) -> None:
+    if pl.local_anchor is None:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, "the planner holds no device state: create it with B, H, S, d")
+
+
 def as_planner_next(pl: AsPlanner, local_now, stream=None):
     """(plan [P,P], is_anchor, ase [P, n_groups]) of the next step."""
+    _check_planner_state(pl)
+    if local_now.dtype != torch.float32 or local_now.shape != pl.local_anchor.shape:
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"local_now must be float32 of the planner's shape {tuple(pl.local_anchor.shape)}, got "
+                      f"{local_now.dtype} {tuple(local_now.shape)}")
     B, H, S, d = local_now.shape
     P = pl.P
     plan = np.zeros(P * P, dtype=np.uint8)
@@ -395,6 +415,15 @@ def as_planner_next(pl: AsPlanner, local_now, stream=None):
 
 
 def as_planner_commit_anchor(pl: AsPlanner, cache: AsCache, lse_full, plan, stream=None):
+    _check_planner_state(pl)
+    want = (cache.B, cache.H, cache.S)
+    if lse_full.dtype != torch.float32 or tuple(lse_full.shape) != want:
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"lse_full must be float32 of the cache's shape {want}, got {lse_full.dtype} "
+                      f"{tuple(lse_full.shape)}")
+    if tuple(pl.local_anchor.shape) != want + (cache.d,):
+        raise AsError(_lib.AS_ERR_INVALID_ARG,
+                      f"the planner's states {tuple(pl.local_anchor.shape)} do not match the cache {want + (cache.d,)}")
     arr = _plan_bytes(plan, pl.P)
     check(LIB.as_planner_commit_anchor(ctypes.byref(pl.struct), ctypes.byref(cache.struct), _dev(lse_full, "lse"),
                                        _dev(pl.local_anchor, "anchor"), arr.ctypes.data, _dev(pl.scratch, "scratch"),

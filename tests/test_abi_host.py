@@ -341,8 +341,33 @@ def test_python_entry_points_check_buffers(api):
         lambda: api.as_plan_drift(torch.zeros(1, 2, 64, 64), torch.zeros(1, 2, 64, 32), 4, torch.zeros(8)),
         lambda: api.as_plan_drift_static(torch.zeros(1, 2, 64, 64), torch.zeros(1, 2, 64, 64).double(), 4),
     ]
+    # inputs of another shape than the cache's: the library would index them with the cache's sizes
+    for qq in [torch.zeros(1, 2, 32, 64, dtype=torch.bfloat16), torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)]:
+        for fn in [lambda: api.as_step(cache, qq, qq, qq, plan, 0),
+                   lambda: api.as_step_local(cache, qq, qq, qq, plan, 0, torch.zeros(qq.shape), torch.zeros(qq.shape[:3]))]:
+            with pytest.raises(api.AsError) as ei:
+                fn()
+            assert "the cache's shape" in str(ei.value)
     for k, fn in enumerate(bad_cases):
         with pytest.raises(api.AsError) as ei:
             fn()
         assert ei.value.status == _lib.AS_ERR_INVALID_ARG, (k, str(ei.value))
         assert "float32" in str(ei.value), (k, str(ei.value))  # not the later device-pointer check
+
+
+def test_planner_entry_points_check_shapes(api):
+    """as_planner_next and as_planner_commit_anchor read the planner's anchor
+    states with the caller's or the cache's sizes: mismatches are refused."""
+    import torch
+    pl = api.AsPlanner(4, 1, 0.5, 0.1, 1, 2, 64, 64, device="cpu")
+    cache = api.AsCache.host_only(1, 2, 64, 64, 4)
+    other = api.AsCache.host_only(1, 2, 128, 64, 4)
+    plan = np.ones((4, 4), np.uint8)
+    for fn in [lambda: api.as_planner_next(pl, torch.zeros(1, 2, 32, 64)),
+               lambda: api.as_planner_next(pl, torch.zeros(1, 2, 64, 64, dtype=torch.float64)),
+               lambda: api.as_planner_commit_anchor(pl, cache, torch.zeros(1, 2, 32), plan),
+               lambda: api.as_planner_commit_anchor(pl, other, torch.zeros(1, 2, 128), plan),
+               lambda: api.as_planner_next(api.AsPlanner(4, 1, 0.5, 0.1), torch.zeros(1, 2, 64, 64))]:
+        with pytest.raises(api.AsError) as ei:
+            fn()
+        assert "must be float32" in str(ei.value) or "do not match" in str(ei.value) or "no device state" in str(ei.value)
