@@ -168,7 +168,9 @@ as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step,
  * entry.  h_hit / h_age (may be NULL) as in as_plan_resolve.  The plan is
  * checked before any launch: on AS_ERR_CACHE_MISS or AS_ERR_INVALID_ARG
  * nothing is launched and the cache is unchanged.  The cache must have been
- * initialised for the same B, H, S, d, P.  The call neither allocates nor
+ * initialised for the same B, H, S, d, P: q, k, v are read and out, lse
+ * written with the cache's sizes, which the library cannot check against the
+ * caller's buffers (the Python binding does).  The call neither allocates nor
  * synchronises, so it can be captured in a CUDA graph: a replay repeats the
  * device work with the captured plan and pointers, while the host
  * bookkeeping (checks, hit/age, t_c, member) happens once, at the captured
