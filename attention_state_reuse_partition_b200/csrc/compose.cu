@@ -237,9 +237,11 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
     };
     // the fp32 sources (composite, local state) lead the list
     const int nf = (a.nsrc[i] > 0 && list[0] < 0) + (a.nsrc[i] > 1 && list[1] < 0);
-    // measured: bf16 planes (half the bytes per load) gain from two sources'
-    // loads in flight, fp32 planes do not
-    compose_rows<D, E, sizeof(E) == 2 ? 2 : 1>(row0, nr, a.nsrc[i], nf, src, a.out, a.lse, lane);
+    // measured: bf16 planes (half the bytes per load) gain from four
+    // sources' loads in flight (496 against 582 us per step compose with
+    // two, although the d = 128 instance then spills about 180 bytes at the
+    // two-CTA register cap); fp32 planes gain nothing from a second
+    compose_rows<D, E, sizeof(E) == 2 ? 4 : 1>(row0, nr, a.nsrc[i], nf, src, a.out, a.lse, lane);
   }
 }
 
