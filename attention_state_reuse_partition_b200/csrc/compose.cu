@@ -201,7 +201,8 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_strided_kernel(const __
   for (long long b = gw; b < nblk; b += stride) {
     const long long row0 = b * RB;
     const int nr = static_cast<int>(min(static_cast<long long>(RB), a.rows - row0));
-    compose_rows<D, float, 2>(row0, nr, a.n_states, 0, src, a.out, a.lse, lane);
+    // three sources' loads in flight: measured 6.95 against 6.90 TB/s with two
+    compose_rows<D, float, 3>(row0, nr, a.n_states, 0, src, a.out, a.lse, lane);
   }
 }
 
