@@ -192,6 +192,13 @@ as_status run_drift(const float* now, const float* anchor, int B, int H, int S, 
   return AS_OK;
 }
 
+// the drift reduction reads both tensors with 16-byte loads
+as_status check_drift_inputs(const float* now, const float* anchor) {
+  if (!aligned16(now) || !aligned16(anchor))
+    return fail(AS_ERR_INVALID_ARG, "local-state tensors must be 16-byte aligned");
+  return AS_OK;
+}
+
 as_status check_planner(const as_planner* pl) {
   if (!pl || pl->magic != PLANNER_MAGIC) return fail(AS_ERR_INVALID_ARG, "planner not initialised by as_planner_init");
   return AS_OK;
@@ -536,6 +543,7 @@ as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (!now || !anchor || !h_drift || !h_norm) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_drift_inputs(now, anchor)) != AS_OK) return s;
   if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;
   std::vector<double> sums(static_cast<size_t>(P) * 2);
@@ -554,6 +562,7 @@ as_status as_plan_drift_static(const float* now, const float* anchor, int B, int
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (!now || !anchor || !h_drift || !h_norm) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_drift_inputs(now, anchor)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;
   double* scratch = nullptr;
   size_t capacity = 0;
@@ -606,6 +615,7 @@ as_status as_planner_next(as_planner* pl, const float* local_now, float* local_a
   const int P = pl->P;
   if ((s = check_shape(B, H, S, d, P)) != AS_OK) return s;
   if (!local_now || !local_anchor || !h_plan || !h_is_anchor) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_drift_inputs(local_now, local_anchor)) != AS_OK) return s;
   if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -653,6 +663,7 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
   if (c->g != pl->g)
     return fail(AS_ERR_INVALID_ARG, "cache groups of %d partitions, planner groups of %d", c->g, pl->g);
   if (!lse_full || !local_anchor || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if ((s = check_drift_inputs(local_anchor, local_anchor)) != AS_OK) return s;
   const int B = c->B, H = c->H, S = c->S, d = c->d, n = S / P;
   if ((s = check_scratch(scratch, scratch_bytes, B, H, P)) != AS_OK) return s;
   if ((s = check_device()) != AS_OK) return s;

@@ -263,7 +263,8 @@ as_status as_local_states(const void* q, const void* k, const void* v, as_dtype 
 
 /* For every partition i: h_drift[i] = ||now_i - anchor_i||_F and h_norm[i] =
  * ||anchor_i||_F over its rows (all b, h, d), reduced in fp64 in a fixed
- * order.  now, anchor [B,H,S,d] fp32 device.  Uses `scratch`; synchronises
+ * order.  now, anchor [B,H,S,d] fp32 device, 16-byte aligned (read with
+ * 16-byte loads; AS_ERR_INVALID_ARG otherwise).  Uses `scratch`; synchronises
  * `stream` (the results are host values). */
 as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int S, int d, int P, void* scratch,
                         size_t scratch_bytes, double* h_drift, double* h_norm, void* stream);
@@ -282,6 +283,10 @@ as_status as_plan_drift(const float* now, const float* anchor, int B, int H, int
  *   sizes in as_last_error().
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is kept for the life of the process: after cudaDeviceReset
+ *   on a device (which unloads the library's device code there), do not
+ *   call this entry point on that device again in the same process.
+ *   local-state pointers must be 16-byte aligned (AS_ERR_INVALID_ARG).
  *   Every call uses the same array and leaves its contents behind; each call
  *   writes every slot it reads, so nothing has to be cleared.  Calls that
  *   overlap on the GPU (different streams, or different host threads on one
@@ -301,7 +306,8 @@ as_status as_plan_select_grouped(const double* h_ase, int P, int g, int window, 
  * local_anchor [B,H,S,d]: the planner's copy of the anchor's local states,
  * overwritten (stream-ordered copy) when this step becomes an anchor.  Writes
  * h_plan [P*P], *h_is_anchor, and h_ase [P*n_groups] (may be NULL; zeros at
- * anchors).  Synchronises `stream`. */
+ * anchors).  local_now and local_anchor must be 16-byte aligned
+ * (AS_ERR_INVALID_ARG otherwise).  Synchronises `stream`. */
 as_status as_planner_next(as_planner* pl, const float* local_now, float* local_anchor, int B, int H, int S, int d,
                           void* scratch, size_t scratch_bytes, uint8_t* h_plan, int* h_is_anchor, double* h_ase,
                           void* stream);
@@ -309,8 +315,8 @@ as_status as_planner_next(as_planner* pl, const float* local_now, float* local_a
 /* After an anchor step (the as_step that used the anchor plan h_plan):
  * measure w and alpha for every entry (pair or group) the plan stored, from
  * the cache (fp32 or bf16 entries), the step's composed LSE lse_full [B,H,S]
- * and local_anchor.  The cache's group size must be the planner's
- * (AS_ERR_INVALID_ARG otherwise).  Synchronises. */
+ * and local_anchor (16-byte aligned).  The cache's group size must be the
+ * planner's (AS_ERR_INVALID_ARG otherwise).  Synchronises. */
 as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const float* lse_full,
                                    const float* local_anchor, const uint8_t* h_plan, void* scratch,
                                    size_t scratch_bytes, void* stream);

@@ -358,7 +358,8 @@ def frob(x):
 
 def scale_ratios(out_pairs, i):
     """alpha(i, j) = ||OUT_ij|| / ||OUT_ii|| for one query partition i;
-    out_pairs [P, ...rows, d]."""
+    out_pairs is a sequence of P states' OUT ([...rows, d] each), entry i the
+    local state (Eq. 9)."""
     norms = np.array([frob(o) for o in out_pairs])
     return norms / norms[i]
 
@@ -453,11 +454,13 @@ def planner_commit_anchor(pl, cache, lse_full, rows_of, n):
     for i in range(P):
         sel = rows_of(i)
         local = pl.local_anchor[..., i * n:(i + 1) * n, :]
-        local_norm = frob(local)
+        lse_i = np.asarray(lse_full)[..., sel]
         for G in range(n_groups(P, pl.g)):
             if (i, G) not in cache.entry or cache.t_c[i, G] < 0:
                 continue
             o, l = cache.entry[(i, G)]
-            pl.w[i, G] = float(np.mean(np.exp(np.asarray(l) - np.asarray(lse_full)[..., sel])))
-            pl.alpha[i, G] = frob(o) / local_norm
+            # Eq. 8 and Eq. 9 for the one entry: the entry against the
+            # composed LSE, and its norm against the local state's
+            pl.w[i, G] = float(anchor_weights(np.asarray(l)[None], lse_i)[0])
+            pl.alpha[i, G] = float(scale_ratios([local, o], 0)[1])
     pl.has_anchor = True

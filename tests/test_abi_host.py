@@ -371,3 +371,38 @@ def test_planner_entry_points_check_shapes(api):
         with pytest.raises(api.AsError) as ei:
             fn()
         assert "must be float32" in str(ei.value) or "do not match" in str(ei.value) or "no device state" in str(ei.value)
+
+
+def test_drift_entry_points_reject_misaligned_local_states(api):
+    """The drift reduction reads the local-state tensors with 16-byte loads:
+    every entry point that feeds it refuses a pointer off that boundary on the
+    host (a view whose storage offset is not a multiple of four floats), so no
+    kernel ever sees it."""
+    from attention_state_reuse_partition_b200 import _lib
+    L = _lib.LIB
+    p, bad = 1 << 20, (1 << 20) + 4
+    B, H, S, d, P = 1, 2, 64, 64, 4
+    h2 = (ctypes.c_double * P)()
+    h3 = (ctypes.c_double * P)()
+    plan = np.ones((P, P), np.uint8)
+    pl = api.AsPlanner(P, 1, 0.5, 0.1)
+    cache = api.AsCache.host_only(B, H, S, d, P)
+    is_anchor = ctypes.c_int(0)
+    calls = {
+        "as_plan_drift now": lambda: L.as_plan_drift(bad, p, B, H, S, d, P, p, 1 << 30, h2, h3, None),
+        "as_plan_drift anchor": lambda: L.as_plan_drift(p, bad, B, H, S, d, P, p, 1 << 30, h2, h3, None),
+        "as_plan_drift_static now": lambda: L.as_plan_drift_static(bad, p, B, H, S, d, P, h2, h3, None),
+        "as_plan_drift_static anchor": lambda: L.as_plan_drift_static(p, bad, B, H, S, d, P, h2, h3, None),
+        "as_planner_next now": lambda: L.as_planner_next(ctypes.byref(pl.struct), bad, p, B, H, S, d, p, 1 << 30,
+                                                         plan.ctypes.data, ctypes.byref(is_anchor), None, None),
+        "as_planner_next anchor": lambda: L.as_planner_next(ctypes.byref(pl.struct), p, bad, B, H, S, d, p,
+                                                            1 << 30, plan.ctypes.data, ctypes.byref(is_anchor),
+                                                            None, None),
+        "as_planner_commit_anchor": lambda: L.as_planner_commit_anchor(ctypes.byref(pl.struct),
+                                                                       ctypes.byref(cache.struct), p, bad,
+                                                                       plan.ctypes.data, p, 1 << 30, None),
+    }
+    for name, call in calls.items():
+        st, msg = _status(call)
+        assert st == _lib.AS_ERR_INVALID_ARG, (name, st, msg)
+        assert "16-byte aligned" in msg, (name, msg)

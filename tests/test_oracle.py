@@ -458,10 +458,10 @@ def pin_planner_trajectory(o):
 
 
 def pin_planner_group_weights(o):
-    """Grouped anchor statistics: the weight of a group entry is the sum of
-    its members' weights (exp of a composed LSE is the sum of the members'
-    exps), computed here from scipy log-sum-exps of the raw scores; alpha is
-    the Frobenius-norm ratio of the group's composed OUT."""
+    """Grouped anchor weights: the weight of a group entry is the sum of its
+    members' weights (exp of a composed LSE is the sum of the members' exps),
+    computed here from scipy log-sum-exps of the raw scores.  The scale
+    ratios of the commit path are pinned by pin_planner_commit_closed_form."""
     r = _rng(35)
     B, H, S, d, P, g = 1, 2, 48, 8, 6, 2
     n = S // P
@@ -486,6 +486,68 @@ def pin_planner_group_weights(o):
             w_sum = sum(float(np.mean(np.exp(scipy.special.logsumexp(sc[..., rows, j * n:(j + 1) * n], axis=-1)
                                              - full[..., rows]))) for j in remote)
             _close(pl.w[i, G], w_sum, 1e-12, f"group weight ({i},{G})")
+
+
+def _scaled_copies(seed, B, H, n, d, c, scale):
+    """Q random; every KV partition holds the same keys k0, and partition j
+    the values c_j * v0.  Then every pair (i, j) has the same scores, so
+    OUT_ij = c_j * A_i with A_i = softmax(scale q_i k0^T) v0 and every LSE_ij
+    is the same: the composed LSE is LSE_ij + ln P."""
+    r = _rng(seed)
+    P = len(c)
+    q = r.normal(size=(B, H, P * n, d))
+    k0 = r.normal(size=(B, H, n, d))
+    v0 = r.normal(size=(B, H, n, d))
+    k = np.concatenate([k0] * P, axis=-2)
+    v = np.concatenate([cj * v0 for cj in c], axis=-2)
+    return q, k, v
+
+
+def pin_planner_commit_closed_form(o):
+    """Anchor statistics and ASE in closed form (DiTango review, Axiom &
+    Free-Parameter Ledger: Eq. 8 importance, Eq. 9 scale ratio
+    alpha(i) = ||AS_ta(i)|| / ||AS_ta(i_loc)|| at the anchor, Eq. 10 and 7).
+
+    With the inputs of _scaled_copies, OUT_ij = c_j * A_i and all LSE_ij are
+    equal, so at the anchor w(i,j) = 1/P and alpha(i,j) = |c_j| / |c_i| for
+    every stored pair.  A group entry of members M composes equal-LSE states,
+    so its OUT is mean_{j in M}(c_j) * A_i: w(i,G) = |M| / P and
+    alpha(i,G) = |mean c_M| / |c_i|.  A local state shifted by the constant s_i
+    has drift D(i) = |s_i| sqrt(#elements), so ASE(i,G) = w * alpha * D(i)."""
+    B, H, n, d, scale = 1, 2, 6, 8, 0.35
+    c = [1.0, -2.0, 0.5, 3.0, -0.25]
+    P = len(c)
+    q, k, v = _scaled_copies(40, B, H, n, d, c, scale)
+    shift = np.array([0.01, 0.02, 0.005, 0.03, 0.015])
+    for g in (1, 2):
+        pl = o.Planner(P, window=0, reuse_ratio=0.5, eps_local=1e9, g=g)
+        cache = o.StateCache(P, g)
+        local = np.concatenate([o.attention_state(q[..., i * n:(i + 1) * n, :], k[..., i * n:(i + 1) * n, :],
+                                                  v[..., i * n:(i + 1) * n, :], scale)[0] for i in range(P)],
+                               axis=-2)
+        plan0, anchor0, _, _ = o.planner_next(pl, local, n)
+        assert anchor0
+        _, lse0, _, _ = o.step(cache, q, k, v, plan0, 0, scale)
+        o.planner_commit_anchor(pl, cache, lse0, lambda i: np.arange(i * n, (i + 1) * n), n)
+        NG = (P + g - 1) // g
+        want_w = np.zeros((P, NG))
+        want_a = np.zeros((P, NG))
+        for i in range(P):
+            for G in range(NG):
+                members = [j for j in range(G * g, min((G + 1) * g, P)) if j != i]
+                if not members:
+                    continue
+                want_w[i, G] = len(members) / P
+                want_a[i, G] = abs(sum(c[j] for j in members) / len(members)) / abs(c[i])
+        _close(pl.w, want_w, 1e-12, f"anchor weights, g={g}")
+        _close(pl.alpha, want_a, 1e-12, f"anchor scale ratios, g={g}")
+        now = local.copy()
+        for i in range(P):
+            now[..., i * n:(i + 1) * n, :] += shift[i]
+        _, anchor1, drift1, a1 = o.planner_next(pl, now, n)
+        assert not anchor1
+        _close(drift1, shift * math.sqrt(B * H * n * d), 1e-12, f"drift of constant shifts, g={g}")
+        _close(a1, want_w * want_a * (shift * math.sqrt(B * H * n * d))[:, None], 1e-12, f"ASE, g={g}")
 
 
 def pin_planner_select_grouped(o):
@@ -529,7 +591,8 @@ PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_for
         pin_planner_weights, pin_planner_ratios, pin_planner_drift, pin_planner_select, pin_planner_trajectory,
         pin_round_bf16, pin_plan_grouped_golden, pin_step_grouped_identical, pin_step_grouped_mixed,
         pin_step_bf16_cache,
-        pin_planner_group_weights, pin_planner_select_grouped, pin_planner_trajectory_grouped]
+        pin_planner_group_weights, pin_planner_select_grouped, pin_planner_trajectory_grouped,
+        pin_planner_commit_closed_form]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -543,7 +606,8 @@ def test_oracle_passes_pin(pin):
 
 _orig = {name: getattr(as_oracle, name) for name in
          ("attention_state", "compose", "compose_pair", "resolve_plan", "step", "partition_bounds",
-          "anchor_weights", "scale_ratios", "local_drift", "select_plan", "ase", "round_bf16", "n_groups")}
+          "anchor_weights", "scale_ratios", "local_drift", "select_plan", "ase", "round_bf16", "n_groups",
+          "planner_commit_anchor")}
 
 
 def _m_no_normalise(q, k, v, scale):
@@ -687,6 +751,12 @@ def _m_ase_no_alpha(w, alpha, drift):
     return _orig["ase"](w, np.ones_like(np.asarray(alpha, dtype=np.float64)), drift)
 
 
+def _m_commit_alpha_inverted(pl, cache, lse_full, rows_of, n):
+    _orig["planner_commit_anchor"](pl, cache, lse_full, rows_of, n)
+    pl.alpha = np.where(pl.alpha > 0, 1.0 / np.where(pl.alpha > 0, pl.alpha, 1.0), 0.0)
+
+
+
 MUTANTS = {
     "attention_state: OUT not normalised": ("attention_state", _m_no_normalise),
     "attention_state: LSE without the scale": ("attention_state", _m_lse_unscaled),
@@ -712,6 +782,7 @@ MUTANTS = {
     "round_bf16: no rounding": ("round_bf16", _m_bf16_not_rounded),
     "n_groups: drops the short last group": ("n_groups", _m_groups_floor),
     "select_plan: a reused group takes its window members too": ("select_plan", _m_select_group_window),
+    "planner_commit_anchor: inverted scale ratio": ("planner_commit_anchor", _m_commit_alpha_inverted),
 }
 
 
