@@ -97,7 +97,7 @@ def _load() -> ctypes.CDLL:
     lib.as_device_status.restype = c_int
     lib.as_device_status.argtypes = [vp, ctypes.POINTER(u32)]
     lib.as_debug_timeout_probe.restype = c_int
-    lib.as_debug_timeout_probe.argtypes = [u32, vp]
+    lib.as_debug_timeout_probe.argtypes = [u32, u32, vp]
     dbl = ctypes.c_double
     lib.as_planner_init.restype = c_int
     lib.as_planner_init.argtypes = [ctypes.POINTER(AsPlannerStruct), c_int, c_int, dbl, dbl]

@@ -449,5 +449,7 @@ def as_debug_exp2(x, mode: int = 0, stream=None):
     return y
 
 
-def as_debug_timeout_probe(poll_budget: int = 64, stream=None) -> None:
-    check(LIB.as_debug_timeout_probe(int(poll_budget), _stream_ptr(stream)))
+def as_debug_timeout_probe(poll_budget: int = 64, limit_ns: int = 4_000_000_000, stream=None) -> None:
+    """One wait on a barrier that nothing completes, bounded by `poll_budget`
+    try_wait rounds or `limit_ns` nanoseconds of GPU time."""
+    check(LIB.as_debug_timeout_probe(int(poll_budget), int(limit_ns), _stream_ptr(stream)))

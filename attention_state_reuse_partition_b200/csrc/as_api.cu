@@ -95,7 +95,6 @@ void base_launch(asp::AttnLaunch& L, const void* q, const void* k, const void* v
   L.P = P;
   L.n = S / P;
   L.scale = scale;
-  L.poll_budget = 1u << 24;
 }
 
 // bit mask of the members of group (i, G) that carry plan code `code`
@@ -474,10 +473,12 @@ as_status as_device_status(void* stream, uint32_t* h_bits) {
   return ok();
 }
 
-as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream) {
+as_status as_debug_timeout_probe(uint32_t poll_budget, uint32_t limit_ns, void* stream) {
+  if (poll_budget < 1) return fail(AS_ERR_INVALID_ARG, "poll_budget must be >= 1");
+  if (limit_ns > 4000000000u) return fail(AS_ERR_INVALID_ARG, "limit_ns must be <= 4e9");
   as_status s = check_device();
   if (s != AS_OK) return s;
-  cudaError_t e = asp::launch_timeout_probe(poll_budget, static_cast<cudaStream_t>(stream));
+  cudaError_t e = asp::launch_timeout_probe(poll_budget, limit_ns, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "timeout probe launch");
   return ok();
 }

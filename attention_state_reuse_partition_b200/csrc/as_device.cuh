@@ -1,10 +1,11 @@
 // Device-side helpers shared by the sm_100a kernels: bounded mbarrier waits,
 // TMA tile loads, tcgen05 (TMEM / UMMA) wrappers and the per-CTA KV schedule.
 //
-// Every wait on an mbarrier is bounded.  When the poll budget runs out the
-// waiting thread records AS_DEVERR_TIMEOUT in the device error word, raises a
-// CTA-local abort flag and returns false; every other wait in the CTA sees the
-// flag and returns as well, so the CTA drains and exits instead of hanging.
+// Every wait on an mbarrier is bounded in time (the GPU's %globaltimer, in
+// nanoseconds).  When the limit runs out the waiting thread records
+// AS_DEVERR_TIMEOUT in the device error word, raises a CTA-local abort flag and
+// returns false; every other wait in the CTA sees the flag and returns as
+// well, so the CTA drains and exits instead of hanging.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -77,19 +78,41 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 #define ASP_TEST_FIRST 1
 #endif
 
+// low 32 bits of the GPU's %globaltimer (nanoseconds); differences of up to
+// 4.29 s are exact in unsigned arithmetic
+__device__ __forceinline__ uint32_t global_ns32() {
+  uint32_t t;
+  asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+  return t;
+}
+
+// The bound of every wait in the kernels: 1 s of GPU time.
+constexpr uint32_t KERNEL_WAIT_NS = 1000000000u;
+
 // Waits until the phase with the given parity has completed.  Returns false
-// (after flagging) when the budget runs out or another thread of the CTA has
-// already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag, uint32_t budget) {
+// (after flagging) when `limit_ns` nanoseconds have passed, when COUNT_POLLS
+// and `polls` rounds of try_wait have come back empty, or when another thread
+// of the CTA has already aborted.  The clock is read only once a try_wait has
+// come back empty, so a wait that succeeds at once costs nothing extra.  The
+// kernels wait without a poll count; the test hook counts polls as well.
+template <bool COUNT_POLLS>
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint32_t polls, uint32_t limit_ns) {
   if (ASP_TEST_FIRST && mbar_test_wait(bar, parity)) return true;
-  for (uint32_t it = 0; it < budget; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t t0 = global_ns32();
+  for (uint32_t it = 1; !COUNT_POLLS || it < polls; ++it) {
     if (*abort_flag) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns32() - t0 > limit_ns) break;
   }
   raise_dev_error(AS_DEVERR_TIMEOUT);
   *abort_flag = 1;
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait_bounded<false>(bar, parity, abort_flag, 0u, KERNEL_WAIT_NS);
 }
 
 // ---------------------------------------------------------------------------

@@ -43,7 +43,6 @@ struct AttnLaunch {
   int dst_bf16;
   int dst_rows, dst_row0;
   long long dst_plane_out, dst_plane_lse;
-  unsigned int poll_budget;
 };
 
 // compose of N states per row with strided state storage (as_compose)
@@ -91,7 +90,7 @@ cudaError_t launch_anchor_stats(const void* cache_out, bool out_bf16, const floa
 cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st);
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st);
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st);
-cudaError_t launch_timeout_probe(unsigned int poll_budget, cudaStream_t st);
+cudaError_t launch_timeout_probe(unsigned int polls, unsigned int ns, cudaStream_t st);
 cudaError_t launch_exp2_probe(const float* x, float* y, long long n, int mode, cudaStream_t st);
 cudaError_t read_and_clear_dev_error(unsigned int* bits, cudaStream_t st);
 

@@ -155,17 +155,20 @@ __device__ int count_tiles(const KvSchedule& s) {
   return n;
 }
 
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint32_t budget) {
-  for (uint32_t it = 0; it < budget; ++it)
+// a wait for work already in flight (copies, MMAs) before the CTA exits;
+// it ignores the abort flag, and is bounded in time like every other wait
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t t0 = global_ns32();
+  while (global_ns32() - t0 <= KERNEL_WAIT_NS)
     if (mbar_try_wait(bar, parity)) return true;
   raise_dev_error(AS_DEVERR_TIMEOUT);
   return false;
 }
 
 // all lanes of a warp wait; the result is the same in every lane
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t budget) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, budget);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -188,7 +191,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int block_lo = L.block_row0 + blk * L.block_rows;
   const int q_lo = block_lo + qt * NQ * BM;
   const int q_hi = min(block_lo + L.block_rows, L.S);  // rows at or beyond q_hi are not written
-  const uint32_t budget = L.poll_budget;
 
   if (threadIdx.x == 0) {
     mbar_init(&c.q_full, 1);
@@ -238,7 +240,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int u = 0;
       for (; u <= n_tiles; ++u) {
         const int slot = u % NST;
-        if (!mbar_wait(&c.kv_empty[slot], ((u / NST) & 1) ^ 1, abort_flag, budget)) break;
+        if (!mbar_wait(&c.kv_empty[slot], ((u / NST) & 1) ^ 1, abort_flag)) break;
         const bool has_k = u < n_tiles, has_v = u >= 1;
         mbar_arrive_expect_tx(&c.kv_full[slot], (has_k ? Lay::TILE_BYTES : 0) + (has_v ? Lay::TILE_BYTES : 0));
         if (has_v) {
@@ -256,8 +258,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       // before the CTA may exit, every issued load must have landed
       if (*abort_flag) {
-        drain_wait(&c.q_full, 0, budget);
-        for (int uu = max(0, u - NST); uu < u; ++uu) drain_wait(&c.kv_full[uu % NST], (uu / NST) & 1, budget);
+        drain_wait(&c.q_full, 0);
+        for (int uu = max(0, u - NST); uu < u; ++uu) drain_wait(&c.kv_full[uu % NST], (uu / NST) & 1);
       }
     }
   } else if (warp == 1) {
@@ -288,7 +290,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                        IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
       };
       // unit 0 (K_0) for the first QKs, unit 1 (V_0, K_1) for the first burst
-      bool ok = mbar_wait(&c.q_full, 0, abort_flag, budget) && mbar_wait(&c.kv_full[0], 0, abort_flag, budget);
+      bool ok = mbar_wait(&c.q_full, 0, abort_flag) && mbar_wait(&c.kv_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < NQ; ++t) {
@@ -296,7 +298,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           umma_commit(&c.s_full[t]);
         }
         umma_commit(&c.kv_empty[0]);
-        ok = mbar_wait(&c.kv_full[1 % NST], (1 / NST) & 1, abort_flag, budget);
+        ok = mbar_wait(&c.kv_full[1 % NST], (1 / NST) & 1, abort_flag);
         TileWalk w;
         int j = 0, group = 0;
         for (w.start(&c.sched); w.valid() && ok; w.next(), ++j) {
@@ -306,8 +308,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int t = 0; t < NQ; ++t) {
             // the burst's data (unit j+1) was waited for earlier; here only
             // the softmax handshake, then the 16 MMAs back to back
-            if (first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag, budget)) ok = false;
-            if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag, budget)) ok = false;
+            if (first && group > 0 && !mbar_wait(&c.o_free[t], (group - 1) & 1, abort_flag)) ok = false;
+            if (ok && !mbar_wait(&c.p_full[t], j & 1, abort_flag)) ok = false;
             if (!ok) break;
             tc_fence_after();
             issue_pv(t, j, first);
@@ -319,7 +321,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             } else if (has_next) {
               // data of the next burst, waited for while the other tile's softmax runs
               const int u = j + 2;
-              if (!mbar_wait(&c.kv_full[u % NST], (u / NST) & 1, abort_flag, budget)) {
+              if (!mbar_wait(&c.kv_full[u % NST], (u / NST) & 1, abort_flag)) {
                 ok = false;
                 break;
               }
@@ -329,7 +331,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       // all issued MMAs must be complete before TMEM is released
       umma_commit(&c.drain);
-      drain_wait(&c.drain, 0, budget);
+      drain_wait(&c.drain, 0);
     }
   }
   } else {
@@ -352,7 +354,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const bool last = w.last();
       const int nv = w.nvalid();
       if (first && j > 0) ++group;
-      if (!warp_wait(&c.s_full[t], j & 1, abort_flag, budget)) break;
+      if (!warp_wait(&c.s_full[t], j & 1, abort_flag)) break;
       tc_fence_after();
       float s[BN];
       {
@@ -439,7 +441,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       l = first ? rs : fmaf(l, alpha, rs);
       m = m_use;
       if (last) {
-        if (!warp_wait(&c.o_ready[t], group & 1, abort_flag, budget)) break;
+        if (!warp_wait(&c.o_ready[t], group & 1, abort_flag)) break;
         tc_fence_after();
         // the warp's 32 rows are consecutive in the destination: s_row0 + rr
         const int s_row0 = s_row - lane;
@@ -553,8 +555,8 @@ cudaError_t launch_d(const AttnLaunch& L, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// One thread waits, with a bounded budget, on a barrier that nothing completes.
-__global__ void timeout_probe_kernel(unsigned int budget) {
+// One thread waits, with the given limit, on a barrier that nothing completes.
+__global__ void timeout_probe_kernel(unsigned int polls, unsigned int ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -563,7 +565,7 @@ __global__ void timeout_probe_kernel(unsigned int budget) {
     mbar_fence_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, budget);
+  if (threadIdx.x == 0) mbar_wait_bounded<true>(&bar, 0, &abort_flag, polls, ns);
 }
 
 __global__ void exp2_probe_kernel(const float* x, float* y, long long n, int mode) {
@@ -585,8 +587,8 @@ cudaError_t launch_exp2_probe(const float* x, float* y, long long n, int mode, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_timeout_probe(unsigned int poll_budget, cudaStream_t st) {
-  timeout_probe_kernel<<<1, 32, 0, st>>>(poll_budget);
+cudaError_t launch_timeout_probe(unsigned int polls, unsigned int ns, cudaStream_t st) {
+  timeout_probe_kernel<<<1, 32, 0, st>>>(polls, ns);
   return cudaGetLastError();
 }
 

@@ -12,7 +12,8 @@
 // rows are read with 128-bit loads, one 512-byte row per warp instruction
 // (d = 128), several sources in flight per lane.  Every input byte is read
 // once from HBM (the LSE re-reads of the third pass hit L1) and the output is
-// written once.  Grids are persistent: 148 SMs x 8 CTAs x 8 warps.
+// written once.  Grids are persistent: 8 CTAs of 8 warps per SM of the
+// current device.
 #include "as_device.cuh"
 
 namespace asp {
@@ -20,7 +21,7 @@ namespace {
 
 constexpr int RB = 8;        // rows per warp block
 constexpr int WARPS = 8;     // warps per CTA
-constexpr int SM_COUNT = 148;
+constexpr int CTAS_PER_SM = 8;
 
 template <int D>
 struct Vec;
@@ -246,16 +247,32 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
   }
 }
 
-long long grid_for(long long nblk) {
+// SMs of the current device
+cudaError_t sm_count(int* n) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  return cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+}
+
+// persistent grid: at most CTAS_PER_SM CTAs per SM, fewer when there is less work
+cudaError_t grid_for(long long nblk, unsigned* grid) {
+  int sms = 0;
+  cudaError_t e = sm_count(&sms);
+  if (e != cudaSuccess) return e;
   const long long ctas = (nblk + WARPS - 1) / WARPS;
-  return ctas < SM_COUNT * 8 ? (ctas > 0 ? ctas : 1) : SM_COUNT * 8;
+  const long long cap = static_cast<long long>(sms) * CTAS_PER_SM;
+  *grid = static_cast<unsigned>(ctas < cap ? (ctas > 0 ? ctas : 1) : cap);
+  return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st) {
   const long long nblk = (a.rows + RB - 1) / RB;
-  const unsigned grid = static_cast<unsigned>(grid_for(nblk));
+  unsigned grid = 0;
+  cudaError_t e = grid_for(nblk, &grid);
+  if (e != cudaSuccess) return e;
   if (a.d == 128)
     compose_strided_kernel<128><<<grid, WARPS * 32, 0, st>>>(a);
   else if (a.d == 64)
@@ -267,7 +284,9 @@ cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st) {
 
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st) {
   const long long nblk = static_cast<long long>(a.B) * a.H * a.P * ((a.n + RB - 1) / RB);
-  const unsigned grid = static_cast<unsigned>(grid_for(nblk));
+  unsigned grid = 0;
+  cudaError_t e = grid_for(nblk, &grid);
+  if (e != cudaSuccess) return e;
   if (a.d == 128 && a.cache_bf16)
     compose_plan_kernel<128, __nv_bfloat16><<<grid, WARPS * 32, 0, st>>>(a);
   else if (a.d == 128)

@@ -194,14 +194,22 @@ as_status as_step_local(as_cache* c, const void* q, const void* k, const void* v
 
 /* Synchronise `stream`, then read and clear the device error word that the
  * kernels' bounded waits set.  *h_bits receives the raw bits (may be NULL).
- * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, else AS_OK. */
+ * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, else AS_OK.
+ *   Every wait inside the attention kernel is bounded by 1 s of the GPU's
+ *   %globaltimer.  A CTA whose pipeline stops therefore gives up at most 1 s
+ *   after its wait began, then waits (again at most 1 s each, three at most)
+ *   for the copies and MMAs it already issued, frees its TMEM and exits: the
+ *   launch ends at most about 4 s after the stall, and this call then
+ *   reports AS_ERR_TIMEOUT. */
 as_status as_device_status(void* stream, uint32_t* h_bits);
 
-/* Test hook for failure detection: launches one CTA that waits, with a poll
- * budget of `poll_budget`, on a barrier that nothing completes.  The wait runs
- * out, sets the device error word and the kernel returns; the context stays
- * usable.  Read the outcome with as_device_status. */
-as_status as_debug_timeout_probe(uint32_t poll_budget, void* stream);
+/* Test hook for failure detection: launches one CTA that waits on a barrier
+ * that nothing completes, with the kernels' wait code and a limit of
+ * `poll_budget` rounds of try_wait (>= 1) or `limit_ns` (<= 4e9) nanoseconds
+ * of the GPU's %globaltimer, whichever comes first.  The wait runs out, sets the
+ * device error word and the kernel returns; the context stays usable.  Read
+ * the outcome with as_device_status. */
+as_status as_debug_timeout_probe(uint32_t poll_budget, uint32_t limit_ns, void* stream);
 
 /* ---------------------------------------------------------------------------
  * The anchor-guided planner (DiTango review: Referee Report major comments 1-3

@@ -313,6 +313,28 @@ def test_timeout_is_reported_and_context_survives(api):
     check_f32(out, lse, ref_o, ref_l, "after timeout")
 
 
+def test_timeout_deadline_in_gpu_time(api):
+    """The kernels bound each wait in time, not in polls: a probe with an
+    unlimited poll count and a 20 ms limit gives up after 20 ms of GPU time
+    (%globaltimer) and reports AS_ERR_TIMEOUT; the host sees the launch end
+    within a bounded wall time, and the context still works afterwards."""
+    import time
+    from attention_state_reuse_partition_b200 import _lib
+    assert api.as_device_status() == 0
+    limit_ns = 20_000_000
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    api.as_debug_timeout_probe(0xFFFFFFFF, limit_ns)
+    with pytest.raises(api.AsError) as ei:
+        api.as_device_status()          # synchronises
+    wall = time.perf_counter() - t0
+    assert ei.value.status == _lib.AS_ERR_TIMEOUT
+    assert limit_ns * 1e-9 <= wall < 2.0, wall
+    assert api.as_device_status() == 0
+    x = torch.randn(1 << 10, device="cuda")
+    assert torch.allclose(api.as_debug_exp2(x, 1), torch.exp2(x), rtol=1e-5)
+
+
 # ---------------------------------------------------------------------------
 # the two exp2 evaluations mixed in the softmax, against CUDA's exp2
 # ---------------------------------------------------------------------------

@@ -4,12 +4,13 @@
   tests;
 * the drift and anchor-statistics reductions: on the same random fp32 inputs,
   against float64 NumPy sums (relative 1e-9);
-* a planner trajectory: anchor decisions and plans against the oracle
-  planner.  Floating point decides these integers, so a pair whose oracle ASE
-  lies within a relative band of the selection threshold, or a step whose
-  relative drift lies within the band around eps_local, may legitimately go
-  either way; everything else must match exactly, and the states of query
-  partitions whose plan rows agree must match the oracle."""
+* a planner trajectory: drift and ASE element by element, anchor decisions
+  and plans against the oracle planner.  Floating point decides these
+  integers, so a unit whose oracle ASE lies within a relative band of the
+  selection threshold, or a step whose relative drift lies within the band
+  around eps_local, may legitimately go either way; there the oracle follows
+  the GPU's choice, everything else must match exactly, and every step's
+  states, hit and age are compared with the oracle's under the same plan."""
 import math
 
 import numpy as np
@@ -110,11 +111,43 @@ def test_anchor_statistics(api, g, cache_dt):
             assert abs(pl.alpha[i, G] - a_ref) <= 1e-9 * a_ref, (i, G)
 
 
+# Tolerances of the trajectory comparison.  The GPU's local states and cache
+# entries come from bf16 inputs through the tensor-core path (P rounded to
+# bf16 in the PV product), so a state's OUT differs from the float64 oracle by
+# about 1e-3 relative.  The drift D(i) is the norm of the difference of two
+# such states 0.1 to 0.4 apart (relative), so its relative error is about
+# 1e-3 / 0.1 = 1e-2; w carries the LSE error (exp of <= 1e-3 absolute: 1e-3
+# relative) and alpha the norm error of two states (~2e-3).  ASE = w alpha D
+# then sits within about 1.5e-2; DRIFT_RTOL and ASE_RTOL leave a factor of two.
+DRIFT_RTOL = 2e-2
+ASE_RTOL = 3e-2
+# a decision whose oracle margin is within BAND (relative) may go either way
+BAND = 3e-2
+
+
+def _rel_drift(local, anchor, P, n):
+    return np.array([O.local_drift(local[..., i * n:(i + 1) * n, :], anchor[..., i * n:(i + 1) * n, :])[0]
+                     / O.frob(anchor[..., i * n:(i + 1) * n, :]) for i in range(P)])
+
+
 @pytest.mark.parametrize("g,cache_dt", [(1, "f32"), (4, "bf16")])
 def test_planner_trajectory_against_oracle(api, g, cache_dt):
-    s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16, steps=6)
-    P, n, window, ratio, eps_local = s.P, s.n, 2, 0.6, 0.25
-    BAND = 1e-2
+    """Seven steps of the planner on a small video trajectory (window 2,
+    R = 0.6, eps_local = 0.4: the oracle anchors at steps 0 and 4 with
+    margins of 6% or more and reuses at steps 1-3, 5 and 6).
+
+    At every step: the anchor decision must match unless the oracle's
+    relative drift lies within BAND of eps_local; at every reuse step the
+    drift and the ASE of every unit are compared element by element with the
+    oracle's, and the plan must match except on units whose oracle ASE lies
+    within BAND of the selection threshold, where either choice is valid (the
+    GPU's plan must still reuse exactly floor(R * #units) units).  Wherever
+    the two may legitimately part, the oracle follows the GPU's decision, so
+    the caches never diverge; then both run the step under the same plan and
+    every state, hit and age is compared.  At least three reuse steps must be
+    compared."""
+    s = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16, steps=7)
+    P, n, window, ratio, eps_local = s.P, s.n, 2, 0.6, 0.4
     steps = [(q.cuda(), k.cuda(), v.cuda()) for _, q, k, v in W.video_trajectory(s)]
     cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, g=g, cache_dtype=cache_dt)
     pl = api.AsPlanner(P, window, ratio, eps_local, s.B, s.H, s.S, s.d, g=g)
@@ -123,23 +156,33 @@ def test_planner_trajectory_against_oracle(api, g, cache_dt):
     units = _units(P, g, window)
     NG = units.shape[1]
     member_of = np.array([[j // g for j in range(P)] for _ in range(P)])  # [i, j] -> G
-    anchors = 0
+    reuse_steps = anchors = 0
     for t, (q, k, v) in enumerate(steps):
         qn, kn, vn = f64(q), f64(k), f64(v)
         local, _ = api.as_local_states(q, k, v, P)
         plan, is_anchor, ase = api.as_planner_next(pl, local)
         olocal, _ = _oracle_local(qn, kn, vn, P, s.scale)
+        saved_anchor = None if opl.local_anchor is None else opl.local_anchor.copy()
+        rel = _rel_drift(olocal, saved_anchor, P, n) if opl.has_anchor else None
         oplan, o_anchor, odrift, oase = O.planner_next(opl, olocal, n)
         if t == 0:
             assert is_anchor and o_anchor
-        else:
-            rel = np.array([odrift[i] / O.frob(opl.local_anchor[..., i * n:(i + 1) * n, :]) if not o_anchor else 0
-                            for i in range(P)])
-            if not o_anchor and abs(rel.max() - eps_local) > BAND * eps_local:
-                assert is_anchor == o_anchor, f"anchor decision at step {t}"
         if is_anchor != o_anchor:
-            break  # an ambiguous anchor decision: the two trajectories part here
-        if not is_anchor:
+            assert abs(rel.max() - eps_local) <= BAND * eps_local, f"anchor decision at step {t}"
+            if is_anchor:   # follow the GPU: the oracle anchors too
+                opl.local_anchor = olocal.copy()
+                oplan, oase = O.anchor_plan(P, window), None
+            else:           # follow the GPU: the oracle keeps its anchor
+                opl.local_anchor = saved_anchor
+                oase = O.ase(opl.w, opl.alpha, odrift)
+                oplan = O.select_plan(oase, window, ratio, g)
+        if is_anchor:
+            assert np.array_equal(plan, O.anchor_plan(P, window))
+        else:
+            reuse_steps += 1
+            assert np.allclose(pl.drift, odrift, rtol=DRIFT_RTOL, atol=0), (t, pl.drift, odrift)
+            assert np.allclose(ase[units], oase[units], rtol=ASE_RTOL, atol=0), \
+                (t, float(np.max(np.abs(ase[units] / oase[units] - 1))))
             vals = np.sort(oase[units])
             k_reuse = int(np.floor(ratio * vals.size + 1e-9))
             thr = vals[k_reuse - 1] if k_reuse > 0 else -np.inf
@@ -149,19 +192,16 @@ def test_planner_trajectory_against_oracle(api, g, cache_dt):
             reused_units = sum(bool((plan[i, G * g:(G + 1) * g] == O.PLAN_REUSE).any())
                                for i in range(P) for G in range(NG))
             assert reused_units == k_reuse
+        # both run the GPU's plan: equal to the oracle's but for ambiguous units
         out, lse, hit, age = api.as_step(cache, q, k, v, plan, t)
         torch.cuda.synchronize()
-        same_rows = [i for i in range(P) if np.array_equal(plan[i], oplan[i])]
-        ref_o, ref_l, _, _ = O.step(ocache, qn, kn, vn, oplan, t, s.scale)
-        for i in same_rows:
-            sl = slice(i * n, (i + 1) * n)
-            check_bf16(out[..., sl, :], lse[..., sl], ref_o[..., sl, :], ref_l[..., sl], f"step {t} partition {i}")
+        ref_o, ref_l, ref_hit, ref_age = O.step(ocache, qn, kn, vn, plan, t, s.scale)
+        assert np.array_equal(hit, ref_hit) and np.array_equal(age, ref_age), f"hit/age at step {t}"
+        check_bf16(out, lse, ref_o, ref_l, f"step {t}")
         if is_anchor:
             anchors += 1
             api.as_planner_commit_anchor(pl, cache, lse, plan)
             O.planner_commit_anchor(opl, ocache, ref_l, lambda i: np.arange(i * n, (i + 1) * n), n)
             assert np.allclose(pl.w[units], opl.w[units], rtol=5e-3, atol=0)
             assert np.allclose(pl.alpha[units], opl.alpha[units], rtol=2e-2, atol=0)
-        if len(same_rows) < P:
-            break  # plans differ on an ambiguous unit: the caches part here
-    assert anchors >= 1
+    assert anchors >= 2 and reuse_steps >= 3, (anchors, reuse_steps)
