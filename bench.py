@@ -8,15 +8,23 @@ composition, on the tensor cores.  FLOPs counted: 4*B*H*S*S*d per step (QK^T
 and PV, fresh pairs only).  Inputs are resident in HBM; the L2 is flushed
 (a 256 MiB write) before every timed step, outside the timed events.
 
-Also reported on the same line (same run):
+Also reported on the same line (same run), in fields of the contract:
 * ``e2e``: the same step through the public API from pinned HOST buffers,
   with the host->device copy of Q, K, V and the device->host copy of OUT and
   LSE inside the timed region;
 * ``roofline``: the attention kernel against the measured dense bf16 peak;
-* ``secondary``: the state-compose kernel on the compose-bound workload (GB/s
-  against measured HBM copy bandwidth) and the two-step video reuse workload
-  (fresh TFLOP/s, reuse-compose GB/s, reuse MSE against full attention);
-* ``cpu_baseline``: the float64 oracle on the host cores on a sample of rows.
+  ``roofline.compose`` the state-compose kernel on the compose-bound workload
+  against the measured HBM copy bandwidth; ``roofline.steps`` every reuse
+  workload's step time against its step-level roofline (tensor time of the
+  fresh pairs and HBM time of the bytes the step must move, summed and
+  overlapped), with the reuse MSE against full attention;
+  ``roofline.partition_boundary`` the flux_image step with one state emitted
+  per KV partition (ragged 576-token partitions inside the timed region);
+  ``roofline.locality`` the MSE of dropping a near against a far partition;
+* ``cpu_baseline``: the float64 oracle on the host cores -- the whole
+  flux_image step, and in ``cpu_baseline.legs`` the compose-bound workload and
+  the video workloads on bounded samples of rows and heads (full-step times
+  extrapolated from the sample, labelled as such).
 
 ``--impl reference`` times the float64 oracle instead (the only reference
 implementation of this method available here), on the host cores, on samples
@@ -215,6 +223,89 @@ def cpu_cores():
     return os.cpu_count()
 
 
+class OracleTrajectory:
+    """The float64 oracle stepped beside a GPU trajectory on a bounded sample:
+    a few heads and a seeded sample of query rows in every query partition,
+    against all keys, under the same plans and cache history.  Each step is
+    timed; its full-workload time is extrapolated by the ratio of rows and
+    heads (labelled as extrapolated).  The GPU's states on the sampled rows
+    are compared with the oracle's (max-abs error, reported)."""
+
+    def __init__(self, s, heads, rows_per_partition: int, g: int = 1, cache_dtype: str = "f32"):
+        from oracle import as_oracle as O
+        self.O, self.s, self.heads = O, s, list(heads)
+        self.rows = W.sample_rows(s, rows_per_partition).numpy()
+        self.cache = O.StateCache(s.P, g, cache_dtype)
+        self.records = []
+
+    def step(self, t, q, k, v, plan, out_gpu=None):
+        s, O = self.s, self.O
+        f = lambda x: x[:, self.heads].float().cpu().double().numpy()  # noqa: E731
+        qn, kn, vn = f(q), f(k), f(v)
+        t0 = time.perf_counter()
+        out, lse, _, _ = O.step(self.cache, qn, kn, vn, plan, t, s.scale, rows=self.rows)
+        dt = time.perf_counter() - t0
+        r = self.rows.size // s.P
+        fresh = int((plan != W.PLAN_REUSE).sum())
+        flop = 4.0 * s.B * len(self.heads) * r * s.n * s.d * fresh
+        factor = (s.S / self.rows.size) * (s.H / len(self.heads))
+        rec = {"step": t, "seconds": round(dt, 3), "tflops": flop / dt / 1e12,
+               "extrapolated_full_step_s": round(dt * factor, 1)}
+        if out_gpu is not None:
+            g = out_gpu[:, self.heads][:, :, torch.from_numpy(self.rows).to(out_gpu.device)]
+            rec["gpu_max_abs_err"] = float(np.max(np.abs(g.double().cpu().numpy() - out)))
+        self.records.append(rec)
+        return rec
+
+    def summary(self, name):
+        s = self.s
+        return {"workload": name, "kind": "oracle", "unit": "TFLOP/s",
+                "value": statistics.mean(x["tflops"] for x in self.records[1:] or self.records),
+                "sample": f"{self.rows.size // s.P} query rows in each of the {s.P} query partitions x "
+                          f"{len(self.heads)} of {s.H} heads, all {s.S} keys, every step of the trajectory; "
+                          f"value = fresh FLOPs of the sample / oracle time, averaged over the non-anchor steps; "
+                          f"extrapolated_full_step_s scales the time by rows and heads (extrapolated, not run)",
+                "steps": self.records}
+
+
+def oracle_compose_sample(outs, lses, rows: int):
+    """The oracle's one-pass compose on the first ``rows`` rows of the
+    compose-bound states; returns (seconds, algorithmic bytes of the sample)."""
+    from oracle import as_oracle as O
+    o = outs[:, :rows].double().cpu().numpy()
+    l = lses[:, :rows].double().cpu().numpy()
+    t0 = time.perf_counter()
+    O.compose([(o[k], l[k]) for k in range(o.shape[0])])
+    dt = time.perf_counter() - t0
+    return dt, (o.shape[0] + 1) * rows * (o.shape[2] + 1) * 4
+
+
+def step_roofline(ms: float, fresh_flop: float, hbm_bytes: float, peaks) -> dict:
+    """A step's time against its roofline: the tensor time of its fresh pairs
+    at the measured bf16 peak and the HBM time of the bytes it must move at
+    the measured copy bandwidth, both serialised (sum) and overlapped (max)."""
+    t_tensor = fresh_flop / (peaks["bf16_tflops"] * 1e12) * 1e3
+    t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+    return {"ms": round(ms, 3), "fresh_flop": fresh_flop, "hbm_bytes": hbm_bytes,
+            "t_tensor_ms": round(t_tensor, 3), "t_hbm_ms": round(t_hbm, 3),
+            "bound_serial_ms": round(t_tensor + t_hbm, 3), "bound_overlap_ms": round(max(t_tensor, t_hbm), 3),
+            "frac_of_serial_bound": round((t_tensor + t_hbm) / ms, 4),
+            "frac_of_overlap_bound": round(max(t_tensor, t_hbm) / ms, 4),
+            "fresh_tflops_whole_step": round(fresh_flop / (ms * 1e-3) / 1e12, 1)}
+
+
+def step_hbm_bytes(s, plan, g: int, cache_dtype: str) -> int:
+    """Bytes a step must move at least: Q, K, V once (bf16), the final OUT and
+    LSE once (fp32), every reused cache entry read once and every stored entry
+    written once (entries of the cache's type, LSE fp32)."""
+    P, NG = s.P, (s.P + g - 1) // g
+    entry = s.B * s.H * s.n * (s.d * (2 if cache_dtype == "bf16" else 4) + 4)
+    reused = sum(bool((plan[i, G * g:(G + 1) * g] == W.PLAN_REUSE).any()) for i in range(P) for G in range(NG))
+    stored = sum(bool((plan[i, G * g:(G + 1) * g] == W.PLAN_FRESH_STORE).any()) for i in range(P) for G in range(NG))
+    io = 3 * s.B * s.H * s.S * s.d * 2 + s.B * s.H * s.S * (s.d + 1) * 4
+    return io + (reused + stored) * entry
+
+
 # ---------------------------------------------------------------------------
 # the timed legs
 # ---------------------------------------------------------------------------
@@ -345,8 +436,9 @@ def ncu_compose_rows() -> int:
     return 196608
 
 
-def run_compose(args, device):
-    """Compose-bound workload: 32 fp32 states per row merged into one."""
+def run_compose(args, device, peaks, with_oracle=False):
+    """Compose-bound workload: 32 fp32 states per row merged into one, against
+    the measured HBM copy bandwidth; optionally the oracle on a row sample."""
     from attention_state_reuse_partition_b200 import api
     s = W.spec("compose_bound")
     outs, lses = W.compose_states(s, device=device, rows=args.compose_rows)
@@ -364,17 +456,34 @@ def run_compose(args, device):
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     rows = outs.shape[1]
     nbytes = (s.n_states + 1) * rows * (s.d + 1) * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    rows_full = s.B * s.H * s.S
+    res = {"bound": "hbm", "kernel": "compose_strided_kernel<128>",
+           "workload": f"compose_bound: {rows} rows (B=2 H=24 S=16384) x {s.n_states} fp32 states, d=128",
+           "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "frac": round(gbs / peaks["hbm_gbs"], 4), "ms": round(ms, 4), "bytes": nbytes,
+           "traffic": measured_traffic("compose_strided_kernel<128>", rows / ncu_compose_rows()),
+           "peak_source": f"{peaks['source']} HBM copy"}
+    cpu = None
+    if with_oracle:
+        n = min(rows, args.oracle_compose_rows)
+        dt, ob = oracle_compose_sample(outs, lses, n)
+        cpu = {"workload": "compose_bound", "kind": "oracle", "unit": "GB/s", "value": ob / dt / 1e9,
+               "sample": f"the first {n} of {rows_full} rows, all {s.n_states} states, float64 one-pass compose; "
+                         f"bytes counted as the GPU's (fp32 states read once, output written once)",
+               "seconds": round(dt, 3), "extrapolated_full_s": round(dt * rows_full / n, 1)}
     del outs, lses, out, lse
     torch.cuda.empty_cache()
-    return {"workload": "compose_bound", "ms": ms, "bytes": nbytes, "GB/s": nbytes / (ms * 1e-3) / 1e9}
+    return res, cpu
 
 
-def run_reuse(args, device):
+def run_reuse(args, device, peaks=None, with_oracle=False):
     """Two-step video reuse: anchor step then a reuse step (window 2).
     ``--reuse-heads`` runs fewer heads (a smaller case for profiling);
     ``--reuse-groups`` / ``--reuse-cache`` set the cache's group size and
-    entry type."""
+    entry type.  With the oracle: both steps on a sample of rows and heads."""
     from attention_state_reuse_partition_b200 import api
+    peaks = peaks or load_peaks()
     s = W.spec("video_reuse") if args.reuse_heads is None else W.spec("video_reuse", H=args.reuse_heads)
     g, cdt = args.reuse_groups, args.reuse_cache
     steps = [(q, k, v) for _, q, k, v in W.video_trajectory(s, device=device)]
@@ -402,33 +511,122 @@ def run_reuse(args, device):
     full_o, _ = api.as_partition_attn(q1, k1, v1, s.P, -1, list(range(s.P)))
     torch.cuda.synchronize()
     mse = torch.mean((out - full_o) ** 2).item()
-    entry_bytes = s.B * s.H * s.n * (s.d * (2 if cdt == "bf16" else 4) + 4)  # one (i, G) entry
     NG = (s.P + g - 1) // g
     reused_entries = sum(bool((plans[1][i, G * g:(G + 1) * g] == W.PLAN_REUSE).any())
                          for i in range(s.P) for G in range(NG))
-    reuse_bytes = reused_entries * entry_bytes
+    res = step_roofline(ms, fresh_flops, step_hbm_bytes(s, plans[1], g, cdt), peaks)
+    res.update({"workload": f"video_reuse step 1 (B=1 H={s.H} S={s.S} P={s.P}, window {s.window}), cache groups "
+                            f"of {g}, {cdt} entries",
+                "fresh_pairs": n_fresh, "reused_pairs": n_reuse, "reused_entries": reused_entries,
+                "reuse_mse_vs_full": mse})
+    cpu = None
+    if with_oracle:
+        orc = OracleTrajectory(s, heads=args.oracle_heads[:min(len(args.oracle_heads), s.H)],
+                               rows_per_partition=args.oracle_rows, g=g, cache_dtype=cdt)
+        c = api.AsCache(s.B, s.H, s.S, s.d, s.P, buffer=cache.buffer, g=g, cache_dtype=cdt)
+        for t in range(s.steps):
+            api.as_step(c, *steps[t], plans[t], t, out=out, lse=lse)
+            torch.cuda.synchronize()
+            orc.step(t, *steps[t], plans[t], out_gpu=out)
+        cpu = orc.summary(res["workload"])
     del cache, steps, full_o
     torch.cuda.empty_cache()
-    name = "video_reuse step t" + ("" if (g, cdt, s.H) == (1, "f32", 24) else f" (H={s.H}, g={g}, {cdt} entries)")
-    return {"workload": name, "ms": ms, "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
-            "reused_entries": reused_entries,
-            "fresh_tflops_whole_step": fresh_flops / (ms * 1e-3) / 1e12, "reuse_bytes": reuse_bytes,
-            "reuse_mse_vs_full": mse}
+    return res, cpu
 
 
-def run_video_long(args, device, g=1, cache_dtype="f32"):
+def run_locality(args, device):
+    """Locality of the video_reuse inputs (the trend DiTango's review page
+    reports in its Core claim: dropping the nearest KV partition costs far
+    more than dropping a distant one).  For every query partition i, the MSE
+    against full attention of the state that leaves out KV partition i+1 (or
+    i-1 at the end) and of the one that leaves out i+8 (or i-8)."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec("video_reuse")
+    _, q, k, v = next(iter(W.video_trajectory(s, device=device)))
+    full_o, _ = api.as_partition_attn(q, k, v, s.P, -1, list(range(s.P)))
+    n = s.n
+    near, far = [], []
+    for i in range(s.P):
+        ref = full_o[:, :, i * n:(i + 1) * n]
+        for dist, acc in ((1, near), (8, far)):
+            j = i + dist if i + dist < s.P else i - dist
+            o, _ = api.as_partition_attn(q, k, v, s.P, i, [x for x in range(s.P) if x != j])
+            acc.append(torch.mean((o - ref) ** 2).item())
+    torch.cuda.synchronize()
+    del q, k, v, full_o
+    torch.cuda.empty_cache()
+    m_near, m_far = statistics.mean(near), statistics.mean(far)
+    return {"workload": "video_reuse step 0", "mse_drop_neighbour": m_near, "mse_drop_distance_8": m_far,
+            "ratio": m_near / m_far if m_far > 0 else None,
+            "what": "mean over query partitions of the MSE against full attention when KV partition i+-1, "
+                    "or i+-8, is left out"}
+
+
+def run_boundary(args, device, merged_tflops: float):
+    """flux_image with one state emitted per KV partition, so that the ragged
+    576-token partitions (4.5 key tiles each) are inside the timed region:
+    (a) the attention kernel alone emitting all eight partition states
+    (as_partition_attn, compose=0); (b) an as_step whose plan stores every
+    pair (the same emission, then the step compose of the eight entries).
+    TFLOP/s count the unmasked work only (4*B*H*S*S*d)."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec(WORKLOAD)
+    q, k, v = W.flux_qkv(s, device=device)
+    flops = attn_flops(s)
+    planes = torch.empty((s.P, s.B, s.H, s.S, s.d), device=device)
+    plse = torch.empty((s.P, s.B, s.H, s.S), device=device)
+    cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device)
+    plan = np.full((s.P, s.P), W.PLAN_FRESH_STORE, np.uint8)
+    out = torch.empty((s.B, s.H, s.S, s.d), device=device)
+    lse = torch.empty((s.B, s.H, s.S), device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=device, dtype=torch.float32)
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i, (a, b) in enumerate(ev):
+            flush.fill_(float(i))
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    ms_emit = timed(lambda: api.as_partition_attn(q, k, v, s.P, -1, list(range(s.P)), compose=False,
+                                                  out=planes, lse=plse))
+    ms_step = timed(lambda: api.as_step(cache, q, k, v, plan, 0, out=out, lse=lse))
+    tiles_real = s.P * math.ceil(s.n / 128)
+    tiles_merged = math.ceil(s.S / 128)
+    del q, k, v, planes, plse, cache, out, lse, flush
+    torch.cuda.empty_cache()
+    emit_tf = flops / (ms_emit * 1e-3) / 1e12
+    return {"workload": f"{WORKLOAD}, one state per KV partition (P={s.P} partitions of {s.n} keys)",
+            "attn_emit_ms": round(ms_emit, 4), "attn_emit_tflops": round(emit_tf, 1),
+            "step_store_all_ms": round(ms_step, 4),
+            "step_store_all_tflops": round(flops / (ms_step * 1e-3) / 1e12, 1),
+            "merged_range_tflops": round(merged_tflops, 1),
+            "emit_vs_merged": round(emit_tf / merged_tflops, 4),
+            "key_tiles_per_query_tile": {"per_partition": tiles_real, "merged": tiles_merged},
+            "masked_tile_fraction": round(1 - tiles_merged / tiles_real, 4),
+            "extra_bytes_written": (s.P - 1) * s.B * s.H * s.S * (s.d + 1) * 4}
+
+
+def run_video_long(args, device, g=1, cache_dtype="f32", peaks=None, with_oracle=False):
     """Long video trajectory: an anchor step, then three reuse steps (window 4,
     a seeded 10% of reused pairs forced fresh and stored each step).  With
     g > 1 the cache keeps one composed entry per (query partition, group of g
     KV partitions) and a forced pair refreshes its whole group."""
     from attention_state_reuse_partition_b200 import api
+    peaks = peaks or load_peaks()
     heads = getattr(args, "video_heads", None)
     s = W.spec("video_long") if heads is None else W.spec("video_long", H=heads)
     cache = api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, g=g, cache_dtype=cache_dtype)
     NG = (s.P + g - 1) // g
-    entry_bytes = s.B * s.H * s.n * (s.d * (2 if cache_dtype == "bf16" else 4) + 4)  # one (i, G) entry
     out = torch.empty((s.B, s.H, s.S, s.d), device=device)
     lse = torch.empty((s.B, s.H, s.S), device=device)
+    orc = OracleTrajectory(s, heads=args.oracle_heads[:2], rows_per_partition=args.oracle_rows // 2, g=g,
+                           cache_dtype=cache_dtype) if with_oracle else None
     per_step = []
     last = None
     for t, q, k, v in W.video_trajectory(s, device=device):
@@ -441,14 +639,13 @@ def run_video_long(args, device, g=1, cache_dtype="f32"):
         b.record()
         torch.cuda.synchronize()
         n_fresh = int((plan != W.PLAN_REUSE).sum())
-        n_reuse = int((plan == W.PLAN_REUSE).sum())
-        n_store = int((plan == W.PLAN_FRESH_STORE).sum())
-        ms = a.elapsed_time(b)
         fl = 4.0 * s.B * s.H * n_fresh * s.n * s.n * s.d
-        per_step.append({"step": t, "ms": round(ms, 3), "fresh_pairs": n_fresh, "reused_pairs": n_reuse,
-                         "stored_pairs": n_store, "reused_entries": reused_entries,
-                         "reuse_read_gb": round(reused_entries * entry_bytes / 1e9, 3),
-                         "fresh_tflops_whole_step": round(fl / (ms * 1e-3) / 1e12, 1)})
+        rec = step_roofline(a.elapsed_time(b), fl, step_hbm_bytes(s, plan, g, cache_dtype), peaks)
+        rec.update({"step": t, "fresh_pairs": n_fresh, "reused_pairs": int((plan == W.PLAN_REUSE).sum()),
+                    "stored_pairs": int((plan == W.PLAN_FRESH_STORE).sum()), "reused_entries": reused_entries})
+        per_step.append(rec)
+        if orc is not None:
+            orc.step(t, q, k, v, plan, out_gpu=out)
         last = (q, k, v)
     q, k, v = last
     full_o, _ = api.as_partition_attn(q, k, v, s.P, -1, list(range(s.P)))
@@ -457,12 +654,11 @@ def run_video_long(args, device, g=1, cache_dtype="f32"):
     cache_gb = cache.buffer.numel() / 1e9
     del cache, full_o, out, lse, last, q, k, v
     torch.cuda.empty_cache()
-    name = "video_long (4 steps)" if g == 1 and cache_dtype == "f32" else \
-        f"video_long (4 steps), cache groups of {g} partitions, {cache_dtype} OUT entries"
-    if heads is not None:
-        name += f" with {s.H} heads"
-    return {"workload": name, "g": g, "cache_dtype": cache_dtype, "cache_gb": round(cache_gb, 2),
-            "steps": per_step, "reuse_mse_vs_full_last_step": mse}
+    name = f"video_long (B=1 H={s.H} S={s.S} P={s.P}, window {s.window}, 4 steps), cache groups of {g}, " \
+           f"{cache_dtype} entries"
+    res = {"workload": name, "cache_gb": round(cache_gb, 2), "steps": per_step,
+           "reuse_mse_vs_full_last_step": mse}
+    return res, (orc.summary(name) if orc is not None else None)
 
 
 def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cache_dtype="f32"):
@@ -523,7 +719,7 @@ def main():
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
     ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner",
-                                       "planner_grouped"], default=None,
+                                       "planner_grouped", "boundary", "locality"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
@@ -534,6 +730,13 @@ def main():
     ap.add_argument("--reuse-cache", choices=["f32", "bf16"], default="f32", help="cache entry type of the reuse workload")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device-resident step only (no e2e, CPU baseline or secondary workloads)")
+    ap.add_argument("--no-oracle", action="store_true", help="skip every oracle (CPU baseline) leg")
+    ap.add_argument("--oracle-rows", type=int, default=64,
+                    help="query rows per partition of the oracle's video samples (video_long uses half)")
+    ap.add_argument("--oracle-heads", type=int, nargs="+", default=[0, 13, 23],
+                    help="heads of the oracle's video samples (video_long uses the first two)")
+    ap.add_argument("--oracle-compose-rows", type=int, default=8192,
+                    help="rows of the oracle's compose-bound sample")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -547,10 +750,15 @@ def main():
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if args.only is not None:
-        fn = {"compose": run_compose, "reuse": run_reuse, "video_long": run_video_long,
-              "video_long_grouped": lambda a, dev: run_video_long(a, dev, g=4, cache_dtype="bf16"),
+        peaks = load_peaks()
+        fn = {"compose": lambda a, dev: run_compose(a, dev, peaks)[0],
+              "reuse": lambda a, dev: run_reuse(a, dev, peaks)[0],
+              "video_long": lambda a, dev: run_video_long(a, dev, peaks=peaks)[0],
+              "video_long_grouped": lambda a, dev: run_video_long(a, dev, g=4, cache_dtype="bf16", peaks=peaks)[0],
               "planner": run_planner,
-              "planner_grouped": lambda a, dev: run_planner(a, dev, g=4, cache_dtype="bf16")}[args.only]
+              "planner_grouped": lambda a, dev: run_planner(a, dev, g=4, cache_dtype="bf16"),
+              "boundary": lambda a, dev: run_boundary(a, dev, float("nan")),
+              "locality": run_locality}[args.only]
         print(json.dumps({"only": args.only, **fn(args, device)}))
         return
     if world > 1:
@@ -559,30 +767,43 @@ def main():
                                              device_id=device)
     peaks = load_peaks()
     res, (q, k, v, s) = run_own(args, rank, world, device)
-    secondary = {}
-    if not args.no_secondary and not args.kernel_only and world == 1:
-        comp = run_compose(args, device)
-        comp["frac_of_hbm"] = comp["GB/s"] / peaks["hbm_gbs"]
-        rows_full = W.spec("compose_bound").B * W.spec("compose_bound").H * W.spec("compose_bound").S
-        comp["traffic"] = measured_traffic("compose_strided_kernel<128>", rows_full / ncu_compose_rows())
-        secondary["compose"] = comp
-        secondary["reuse"] = run_reuse(args, device)
-        secondary["video_long"] = run_video_long(args, device)
-        secondary["video_long_grouped"] = run_video_long(args, device, g=4, cache_dtype="bf16")
-        secondary["planner"] = run_planner(args, device)
-        secondary["planner_grouped"] = run_planner(args, device, g=4, cache_dtype="bf16")
-
+    ms = res["ms_max"]
+    achieved = res["flops"] / (res["ms"] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": measured_traffic("attn_tc_kernel<128>"),
+                "kernel": "attn_tc_kernel<128>", "peak_source": f"{peaks['source']} bf16 burst",
+                # the kernel is timed after a second of full load, at the power-capped clock
+                "peak_sustained": peaks["bf16_tflops_sustained"],
+                "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)}
     cpu = None
-    if rank == 0 and world == 1 and not args.kernel_only:
+    legs = {}
+    full = not args.no_secondary and not args.kernel_only and world == 1
+    oracle_on = rank == 0 and world == 1 and not args.kernel_only and not args.no_oracle
+    if oracle_on:
         heads = list(range(s.H))
         dt, fl = oracle_sample(s, q, k, v, s.n, heads)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": f"the whole {WORKLOAD} step (all {s.S} query rows x {s.H} heads, all {s.S} keys), "
                          f"float64, one pass ({dt:.1f} s)"}
+    del q, k, v
+    torch.cuda.empty_cache()
+    if full:
+        roofline["compose"], legs["compose_bound"] = run_compose(args, device, peaks, with_oracle=oracle_on)
+        steps = {}
+        steps["video_reuse"], legs["video_reuse"] = run_reuse(args, device, peaks, with_oracle=oracle_on)
+        a2 = argparse.Namespace(**{**vars(args), "reuse_groups": 4, "reuse_cache": "bf16"})
+        steps["video_reuse_g4_bf16"], _ = run_reuse(a2, device, peaks)
+        steps["video_long"], legs["video_long"] = run_video_long(args, device, peaks=peaks, with_oracle=oracle_on)
+        steps["video_long_g4_bf16"], _ = run_video_long(args, device, g=4, cache_dtype="bf16", peaks=peaks)
+        steps["planner"] = run_planner(args, device)
+        steps["planner_g4_bf16"] = run_planner(args, device, g=4, cache_dtype="bf16")
+        roofline["steps"] = steps
+        roofline["partition_boundary"] = run_boundary(args, device, achieved)
+        roofline["locality"] = run_locality(args, device)
+    if cpu is not None and legs:
+        cpu["legs"] = {k: v for k, v in legs.items() if v is not None}
 
-    ms = res["ms_max"]
-    achieved = res["flops"] / (res["ms"] * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
     line = {
         "metric": METRIC, "value": round(res["value"], 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
@@ -590,20 +811,13 @@ def main():
         "config": {"workload": WORKLOAD_TEXT, "global_batch": world, "seq_len": s.S,
                    "parallelism": f"replicas{world}" if world > 1 else "single", "l2": "flushed (256 MiB write) "
                    "before every timed step"},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": measured_traffic("attn_tc_kernel<128>"),
-                     "kernel": "attn_tc_kernel<128>", "peak_source": f"{peaks['source']} bf16 burst",
-                     # the kernel is timed after a second of full load, at the power-capped clock
-                     "peak_sustained": peaks["bf16_tflops_sustained"],
-                     "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)},
+        "roofline": roofline,
         "e2e": res["e2e"], "clocks": res["clocks"], "gpu_launches": res["gpu_launches"],
     }
     if line["e2e"] is None:
         del line["e2e"]
     if cpu:
         line["cpu_baseline"] = cpu
-    if secondary:
-        line["secondary"] = secondary
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
