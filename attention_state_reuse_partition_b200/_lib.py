@@ -25,7 +25,7 @@ EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as
            "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
            "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static",
            "as_cache_group_bytes", "as_cache_group_init", "as_planner_group_init", "as_plan_select_grouped",
-           "as_step_local")
+           "as_step_local", "as_cache_cp_bytes", "as_cache_cp_init", "as_step_cp")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -38,6 +38,7 @@ class AsCacheStruct(ctypes.Structure):
         ("t_c", ctypes.c_int32 * (AS_MAX_P * AS_MAX_P)),
         ("g", ctypes.c_int), ("n_groups", ctypes.c_int),
         ("member", ctypes.c_uint64 * (AS_MAX_P * AS_MAX_P)),
+        ("q_first", ctypes.c_int), ("q_count", ctypes.c_int),
     ]
 
 
@@ -94,6 +95,14 @@ def _load() -> ctypes.CDLL:
     lib.as_step_local.restype = c_int
     lib.as_step_local.argtypes = [ctypes.POINTER(AsCacheStruct), vp, vp, vp, c_int, c_float, vp, c_int, vp, vp,
                                   vp, vp, vp, vp, vp]
+    lib.as_cache_cp_bytes.restype = sz
+    lib.as_cache_cp_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int]
+    lib.as_cache_cp_init.restype = c_int
+    lib.as_cache_cp_init.argtypes = [ctypes.POINTER(AsCacheStruct), vp, sz, c_int, c_int, c_int, c_int, c_int,
+                                     c_int, c_int, c_int, c_int]
+    lib.as_step_cp.restype = c_int
+    lib.as_step_cp.argtypes = [ctypes.POINTER(AsCacheStruct), vp, vp, vp, c_int, vp, c_int, c_float, vp, c_int,
+                               vp, vp, vp, vp, vp]
     lib.as_device_status.restype = c_int
     lib.as_device_status.argtypes = [vp, ctypes.POINTER(u32)]
     lib.as_debug_timeout_probe.restype = c_int

@@ -18,7 +18,7 @@ __all__ = ["as_partition_attn", "as_compose", "as_cache_bytes", "as_cache_init",
            "as_device_status", "as_debug_timeout_probe", "as_version", "AsCache", "AsError",
            "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE", "AsPlanner", "as_planner_init",
            "as_planner_scratch_bytes", "as_local_states", "as_plan_drift", "as_plan_select", "as_planner_next",
-           "as_planner_commit_anchor", "as_plan_drift_static", "as_step_local"]
+           "as_planner_commit_anchor", "as_plan_drift_static", "as_step_local", "as_cache_cp_bytes", "as_step_cp"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -114,33 +114,44 @@ def as_cache_bytes(B: int, H: int, S: int, d: int, P: int, g: int = 1, cache_dty
     return int(LIB.as_cache_group_bytes(B, H, S, d, P, g, _cache_dt(cache_dtype)))
 
 
+def as_cache_cp_bytes(B: int, H: int, S: int, d: int, P: int, q_count: int, g: int = 1,
+                      cache_dtype=torch.float32) -> int:
+    return int(LIB.as_cache_cp_bytes(B, H, S, d, P, g, _cache_dt(cache_dtype), q_count))
+
+
 class AsCache:
     """A state cache: the C struct plus its device buffer (allocated with
     torch).  ``g``: KV partitions per cache group (one composed entry per
     (query partition, group)); ``cache_dtype``: torch.float32 or
-    torch.bfloat16 for the OUT entries (LSE entries are fp32)."""
+    torch.bfloat16 for the OUT entries (LSE entries are fp32).  ``q_first``,
+    ``q_count``: the query partitions the cache holds entries for (all of
+    them by default; one rank's run for context parallelism, as_step_cp)."""
 
     def __init__(self, B: int, H: int, S: int, d: int, P: int, device="cuda", buffer: Optional[torch.Tensor] = None,
-                 g: int = 1, cache_dtype=torch.float32):
+                 g: int = 1, cache_dtype=torch.float32, q_first: int = 0, q_count: Optional[int] = None):
         dt = _cache_dt(cache_dtype)
-        nbytes = as_cache_bytes(B, H, S, d, P, g, dt)
+        q_count = P if q_count is None else q_count
+        nbytes = as_cache_cp_bytes(B, H, S, d, P, q_count, g, dt)
         if nbytes == 0:
             raise AsError(_lib.AS_ERR_INVALID_ARG, "invalid cache sizes")
         if buffer is None:
             buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.buffer = buffer
         self.struct = AsCacheStruct()
-        check(LIB.as_cache_group_init(ctypes.byref(self.struct), buffer.data_ptr(), buffer.numel(), B, H, S, d, P, g,
-                                      dt))
-        self._set_sizes(B, H, S, d, P, g, dt)
+        check(LIB.as_cache_cp_init(ctypes.byref(self.struct), buffer.data_ptr(), buffer.numel(), B, H, S, d, P, g,
+                                   dt, q_first, q_count))
+        self._set_sizes(B, H, S, d, P, g, dt, q_first, q_count)
 
-    def _set_sizes(self, B, H, S, d, P, g, dt):
+    def _set_sizes(self, B, H, S, d, P, g, dt, q_first=0, q_count=None):
         self.B, self.H, self.S, self.d, self.P, self.g = B, H, S, d, P, g
+        self.q_first, self.q_count = q_first, (P if q_count is None else q_count)
+        self.rows = self.q_count * (S // P)  # query rows per head of the cache's planes
         self.NG = (P + g - 1) // g
         self.cache_dtype = torch.bfloat16 if dt == AS_BF16 else torch.float32
 
     @classmethod
-    def host_only(cls, B: int, H: int, S: int, d: int, P: int, g: int = 1, cache_dtype=torch.float32) -> "AsCache":
+    def host_only(cls, B: int, H: int, S: int, d: int, P: int, g: int = 1, cache_dtype=torch.float32,
+                  q_first: int = 0, q_count: Optional[int] = None) -> "AsCache":
         """A cache struct for host-side plan bookkeeping (as_plan_resolve) on a
         machine without a GPU.  Its planes point at a placeholder address that
         is never dereferenced; it must not be passed to as_step."""
@@ -148,9 +159,10 @@ class AsCache:
         self.buffer = None
         self.struct = AsCacheStruct()
         dt = _cache_dt(cache_dtype)
-        check(LIB.as_cache_group_init(ctypes.byref(self.struct), 1 << 30, as_cache_bytes(B, H, S, d, P, g, dt),
-                                      B, H, S, d, P, g, dt))
-        self._set_sizes(B, H, S, d, P, g, dt)
+        q_count = P if q_count is None else q_count
+        check(LIB.as_cache_cp_init(ctypes.byref(self.struct), 1 << 30, as_cache_cp_bytes(B, H, S, d, P, q_count, g, dt),
+                                   B, H, S, d, P, g, dt, q_first, q_count))
+        self._set_sizes(B, H, S, d, P, g, dt, q_first, q_count)
         return self
 
     def set_t_c(self, t_c) -> None:
@@ -180,6 +192,7 @@ class AsCache:
         host bookkeeping (t_c, member masks) and a host copy of the device
         buffer (synchronises the current stream)."""
         return {"sizes": (self.B, self.H, self.S, self.d, self.P), "g": self.g,
+                "q_first": self.q_first, "q_count": self.q_count,
                 "cache_dtype": "bf16" if self.cache_dtype == torch.bfloat16 else "f32",
                 "t_c": self.t_c, "member": self.member,
                 "buffer": None if self.buffer is None else self.buffer.cpu()}
@@ -188,7 +201,8 @@ class AsCache:
     def from_state_dict(cls, sd: dict, device="cuda") -> "AsCache":
         """A cache restored from state_dict(): same entries and bookkeeping."""
         B, H, S, d, P = sd["sizes"]
-        self = cls(B, H, S, d, P, device=device, g=sd["g"], cache_dtype=sd["cache_dtype"])
+        self = cls(B, H, S, d, P, device=device, g=sd["g"], cache_dtype=sd["cache_dtype"],
+                   q_first=sd.get("q_first", 0), q_count=sd.get("q_count"))
         if sd["buffer"] is None or sd["buffer"].numel() != self.buffer.numel():
             raise AsError(_lib.AS_ERR_INVALID_ARG, "state dict buffer does not match the cache sizes")
         self.buffer.copy_(sd["buffer"])
@@ -197,14 +211,14 @@ class AsCache:
         return self
 
     def planes(self):
-        """Views of the cache planes: OUT [NG,B,H,S,d] (the cache dtype), LSE
-        [NG,B,H,S] (fp32)."""
-        n_out = self.NG * self.B * self.H * self.S * self.d
-        n_lse = self.NG * self.B * self.H * self.S
+        """Views of the cache planes: OUT [NG,B,H,rows,d] (the cache dtype),
+        LSE [NG,B,H,rows] (fp32); rows = S unless the cache is one rank's."""
+        n_out = self.NG * self.B * self.H * self.rows * self.d
+        n_lse = self.NG * self.B * self.H * self.rows
         esz = 2 if self.cache_dtype == torch.bfloat16 else 4
-        out = self.buffer[: n_out * esz].view(self.cache_dtype).view(self.NG, self.B, self.H, self.S, self.d)
+        out = self.buffer[: n_out * esz].view(self.cache_dtype).view(self.NG, self.B, self.H, self.rows, self.d)
         lse = self.buffer[n_out * esz: n_out * esz + n_lse * 4].view(torch.float32).view(
-            self.NG, self.B, self.H, self.S)
+            self.NG, self.B, self.H, self.rows)
         return out, lse
 
 
@@ -274,6 +288,38 @@ def as_step_local(cache: AsCache, q, k, v, plan, step: int, local_out, local_lse
 # ---------------------------------------------------------------------------
 # the anchor-guided planner
 # ---------------------------------------------------------------------------
+
+def as_step_cp(cache: AsCache, q, k_buf, v_buf, kv_slots, plan, step: int, scale: Optional[float] = None,
+               out=None, lse=None, stream=None):
+    """One step on the rank that owns the cache's query partitions: q [B, H,
+    cache.rows, d] holds its query rows, k_buf / v_buf [B, H, kv_rows, d] the
+    KV partitions its plan rows compute (partition j at rows kv_slots[j] * n,
+    -1 = absent; see cp.exchange_kv).  Returns (out, lse, hit, age) for the
+    rank's rows; hit and age are [P, P] with zeros outside them."""
+    want = (cache.B, cache.H, cache.rows, cache.d)
+    if q.dim() != 4 or tuple(q.shape) != want:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, f"q must have shape {want}, got {tuple(q.shape)}")
+    for name, t in (("k_buf", k_buf), ("v_buf", v_buf)):
+        if t.dim() != 4 or t.shape[:2] != q.shape[:2] or t.shape[3] != q.shape[3] or t.dtype != q.dtype \
+                or t.device != q.device or t.shape != k_buf.shape:
+            raise AsError(_lib.AS_ERR_INVALID_ARG,
+                          f"{name} ({tuple(t.shape)}, {t.dtype}) must be [B, H, kv_rows, d] like k_buf, with q's "
+                          f"B, H, d, dtype and device")
+    P = cache.P
+    slots = np.ascontiguousarray(np.asarray(kv_slots, dtype=np.int32).reshape(P))
+    B, H, R, d = q.shape
+    scale = 1.0 / d ** 0.5 if scale is None else scale
+    out = _buf(out, (B, H, R, d), q.device, "out")
+    lse = _buf(lse, (B, H, R), q.device, "lse")
+    arr = _plan_bytes(plan, P)
+    hit = np.zeros(P * P, dtype=np.uint8)
+    age = np.zeros(P * P, dtype=np.int32)
+    check(LIB.as_step_cp(ctypes.byref(cache.struct), _dev(q, "q"), _dev(k_buf, "k_buf"), _dev(v_buf, "v_buf"),
+                         int(k_buf.shape[2]), slots.ctypes.data, _dtype_code(q), float(scale), arr.ctypes.data,
+                         int(step), _dev(out, "out"), _dev(lse, "lse"), hit.ctypes.data, age.ctypes.data,
+                         _stream_ptr(stream)))
+    return out, lse, hit.reshape(P, P), age.reshape(P, P)
+
 
 def as_planner_scratch_bytes(B: int, H: int, P: int) -> int:
     return int(LIB.as_planner_scratch_bytes(B, H, P))

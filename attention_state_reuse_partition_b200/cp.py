@@ -1,0 +1,146 @@
+"""Context parallelism over ranks for the attention-state step.
+
+DiTango (arXiv 2607.15650; review page, Referee Report "Summary": group-wise
+KV transfer and ring-based composition across GPUs; "Core claim": cached
+states stand in for far KV partitions) runs the query partitions of one
+sequence on several GPUs.  Here each rank owns a contiguous run of query
+partitions and the K/V rows of the same partitions.  Before a step a rank
+fetches from the other ranks only the KV partitions that its rows of the plan
+compute fresh (codes 1 and 2); a reused pair moves nothing, because its
+cached state lives on the rank that owns the query partition.  After the
+exchange the rank runs ``as_step_cp`` on its own rows, its own cache and the
+compact K/V buffer.
+
+Everything here is host logic plus point-to-point sends and receives through
+``torch.distributed`` (NCCL on GPUs, gloo on CPU); the arithmetic runs in the
+library's kernels.  No TMA multicast is involved anywhere on this path.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+import torch
+
+PLAN_REUSE = 0
+
+
+@dataclasses.dataclass(frozen=True)
+class CpLayout:
+    """P partitions over `world` ranks: rank r owns the contiguous run
+    ``parts(r)`` of query partitions (and of K/V partitions); the first
+    P % world ranks own one partition more than the others."""
+    P: int
+    world: int
+
+    def __post_init__(self):
+        if self.world < 1 or self.P < self.world:
+            raise ValueError(f"need 1 <= world <= P (P={self.P}, world={self.world})")
+
+    def parts(self, rank: int) -> range:
+        base, extra = divmod(self.P, self.world)
+        lo = rank * base + min(rank, extra)
+        return range(lo, lo + base + (1 if rank < extra else 0))
+
+    def owner(self, j: int) -> int:
+        for r in range(self.world):
+            if j in self.parts(r):
+                return r
+        raise ValueError(f"partition {j} out of [0, {self.P})")
+
+
+def needed_kv(plan, parts: Sequence[int]) -> List[int]:
+    """KV partitions that the rows ``parts`` of the plan compute fresh, sorted."""
+    plan = np.asarray(plan)
+    return sorted({j for i in parts for j in range(plan.shape[1]) if int(plan[i, j]) != PLAN_REUSE})
+
+
+def exchange_plan(plan, layout: CpLayout) -> Dict[Tuple[int, int], List[int]]:
+    """{(src, dst): partitions src sends to dst} for src != dst: the
+    partitions src owns that dst needs."""
+    out = {}
+    for dst in range(layout.world):
+        need = needed_kv(plan, layout.parts(dst))
+        for src in range(layout.world):
+            if src != dst:
+                js = [j for j in need if j in layout.parts(src)]
+                if js:
+                    out[(src, dst)] = js
+    return out
+
+
+def kv_slots(needed: Sequence[int], P: int) -> np.ndarray:
+    """Slot of every KV partition in a rank's compact K/V buffer (int32 [P],
+    -1 = not present): the needed partitions in increasing order."""
+    slots = np.full(P, -1, dtype=np.int32)
+    for s, j in enumerate(sorted(needed)):
+        slots[j] = s
+    return slots
+
+
+def exchange_bytes(plan, layout: CpLayout, B: int, H: int, n: int, d: int, elem_bytes: int) -> Dict[str, int]:
+    """Bytes a step's exchange moves between ranks (K and V), and what an
+    all-gather of every partition would move."""
+    per_part = 2 * B * H * n * d * elem_bytes
+    moved = sum(len(js) for js in exchange_plan(plan, layout).values()) * per_part
+    all_gather = sum(layout.P - len(layout.parts(r)) for r in range(layout.world)) * per_part
+    return {"moved": moved, "all_gather": all_gather}
+
+
+def _rows(t: torch.Tensor, js: Sequence[int], first: int, n: int) -> torch.Tensor:
+    """Rows of partitions js (owned run starting at partition `first`) of a
+    [B, H, rows, d] tensor, concatenated in order, contiguous."""
+    return torch.cat([t[:, :, (j - first) * n:(j - first + 1) * n] for j in js], dim=2).contiguous()
+
+
+def exchange_kv(k_local: torch.Tensor, v_local: torch.Tensor, plan, layout: CpLayout, rank: int, n: int,
+                group=None) -> Tuple[torch.Tensor, torch.Tensor, np.ndarray]:
+    """The exchange of one step on one rank.
+
+    k_local, v_local: [B, H, n * len(parts(rank)), d], the rank's own
+    partitions.  Returns (k_buf, v_buf, slots): [B, H, n * #needed, d] with
+    KV partition j at rows [slots[j] * n, (slots[j] + 1) * n).  Every rank of
+    the group must call this with the same plan (the sends and receives pair
+    up); each message carries all the partitions of one (src, dst) pair, K
+    and V separately."""
+    import torch.distributed as dist
+    mine = layout.parts(rank)
+    need = needed_kv(plan, mine)
+    slots = kv_slots(need, layout.P)
+    B, H, _, d = k_local.shape
+    k_buf = torch.empty((B, H, n * len(need), d), dtype=k_local.dtype, device=k_local.device)
+    v_buf = torch.empty_like(k_buf)
+    for j in need:
+        if j in mine:
+            s = int(slots[j])
+            k_buf[:, :, s * n:(s + 1) * n] = k_local[:, :, (j - mine.start) * n:(j - mine.start + 1) * n]
+            v_buf[:, :, s * n:(s + 1) * n] = v_local[:, :, (j - mine.start) * n:(j - mine.start + 1) * n]
+    pairs = exchange_plan(plan, layout)
+    ops, recvs = [], []
+    for (src, dst), js in sorted(pairs.items()):
+        if src == rank:
+            for t in (k_local, v_local):
+                ops.append(dist.P2POp(dist.isend, _rows(t, js, mine.start, n), dst, group=group))
+        elif dst == rank:
+            bufs = [torch.empty((B, H, n * len(js), d), dtype=k_local.dtype, device=k_local.device)
+                    for _ in range(2)]
+            for b in bufs:
+                ops.append(dist.P2POp(dist.irecv, b, src, group=group))
+            recvs.append((js, bufs))
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+    for js, (kb, vb) in recvs:
+        for x, j in enumerate(js):
+            s = int(slots[j])
+            k_buf[:, :, s * n:(s + 1) * n] = kb[:, :, x * n:(x + 1) * n]
+            v_buf[:, :, s * n:(s + 1) * n] = vb[:, :, x * n:(x + 1) * n]
+    return k_buf, v_buf, slots
+
+
+def gather_kv_local(k: torch.Tensor, v: torch.Tensor, needed: Sequence[int], n: int):
+    """The buffers exchange_kv would produce, built from the full K/V of one
+    process (for a single-GPU stand-in of one rank)."""
+    js = sorted(needed)
+    return _rows(k, js, 0, n), _rows(v, js, 0, n), kv_slots(js, k.shape[2] // n)

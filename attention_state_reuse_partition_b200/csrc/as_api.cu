@@ -95,6 +95,8 @@ void base_launch(asp::AttnLaunch& L, const void* q, const void* k, const void* v
   L.P = P;
   L.n = S / P;
   L.scale = scale;
+  L.S_kv = S;
+  for (int j = 0; j < P; ++j) L.kv_row0[j] = j * (S / P);
 }
 
 // bit mask of the members of group (i, G) that carry plan code `code`
@@ -107,16 +109,20 @@ uint64_t group_mask(const uint8_t* plan, int P, int g, int i, int G, uint8_t cod
 
 // hit / age of a plan against the cache bookkeeping; codes checked first, then
 // groups that mix reuse and store, then misses (never stored, or other members)
+// rows q_first .. q_first + q_count - 1 of the plan belong to the cache's
+// query partitions (all of them unless the cache is one rank's); the other
+// rows are only checked for valid codes, and their hit and age are 0
 as_status resolve(const as_cache* c, const uint8_t* plan, int step, uint8_t* hit, int32_t* age) {
   const int P = c->P, g = c->g, NG = c->n_groups;
+  const int i0 = c->q_first, i1 = c->q_first + c->q_count;
   for (int x = 0; x < P * P; ++x)
     if (plan[x] > AS_PLAN_FRESH_STORE)
       return fail(AS_ERR_INVALID_ARG, "plan[%d][%d] = %d is not 0, 1 or 2", x / P, x % P, plan[x]);
-  for (int i = 0; i < P; ++i)
+  for (int i = i0; i < i1; ++i)
     for (int G = 0; G < NG; ++G)
       if (group_mask(plan, P, g, i, G, AS_PLAN_REUSE) && group_mask(plan, P, g, i, G, AS_PLAN_FRESH_STORE))
         return fail(AS_ERR_INVALID_ARG, "group (%d, %d) of size %d both reuses and stores members", i, G, g);
-  for (int i = 0; i < P; ++i)
+  for (int i = i0; i < i1; ++i)
     for (int G = 0; G < NG; ++G) {
       const uint64_t r = group_mask(plan, P, g, i, G, AS_PLAN_REUSE);
       if (!r) continue;
@@ -127,7 +133,7 @@ as_status resolve(const as_cache* c, const uint8_t* plan, int step, uint8_t* hit
                     static_cast<unsigned long long>(r), static_cast<unsigned long long>(c->member[i * NG + G]));
     }
   for (int x = 0; x < P * P; ++x) {
-    const bool r = plan[x] == AS_PLAN_REUSE;
+    const bool r = plan[x] == AS_PLAN_REUSE && x / P >= i0 && x / P < i1;
     if (hit) hit[x] = r ? 1 : 0;
     if (age) age[x] = r ? step - c->t_c[(x / P) * NG + (x % P) / g] : 0;
   }
@@ -287,27 +293,33 @@ as_status as_compose(const float* outs, const float* lses, int n_states, int64_t
   return ok();
 }
 
-size_t as_cache_group_bytes(int B, int H, int S, int d, int P, int g, as_dtype cache_dt) {
+size_t as_cache_cp_bytes(int B, int H, int S, int d, int P, int g, as_dtype cache_dt, int q_count) {
   if (cache_dt != AS_F32 && cache_dt != AS_BF16) return 0;
-  if (check_shape(B, H, S, d, P) != AS_OK || g < 1 || g > P) return 0;
+  if (check_shape(B, H, S, d, P) != AS_OK || g < 1 || g > P || q_count < 1 || q_count > P) return 0;
   const size_t NG = static_cast<size_t>((P + g - 1) / g);
-  const size_t rows = static_cast<size_t>(B) * H * S;
+  const size_t rows = static_cast<size_t>(B) * H * q_count * (S / P);
   return NG * rows * (static_cast<size_t>(d) * (cache_dt == AS_BF16 ? 2 : 4) + sizeof(float));
+}
+
+size_t as_cache_group_bytes(int B, int H, int S, int d, int P, int g, as_dtype cache_dt) {
+  return as_cache_cp_bytes(B, H, S, d, P, g, cache_dt, P);
 }
 
 size_t as_cache_bytes(int B, int H, int S, int d, int P, as_dtype cache_dt) {
   return as_cache_group_bytes(B, H, S, d, P, 1, cache_dt);
 }
 
-as_status as_cache_group_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, int g,
-                              as_dtype cache_dt) {
+as_status as_cache_cp_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, int g,
+                           as_dtype cache_dt, int q_first, int q_count) {
   if (!c) return fail(AS_ERR_INVALID_ARG, "null cache struct");
   if (cache_dt != AS_F32 && cache_dt != AS_BF16)
     return fail(AS_ERR_INVALID_ARG, "cache dtype %d is not AS_F32 or AS_BF16", static_cast<int>(cache_dt));
   as_status s = check_shape(B, H, S, d, P);
   if (s != AS_OK) return s;
   if (g < 1 || g > P) return fail(AS_ERR_INVALID_ARG, "group size %d outside [1, %d]", g, P);
-  const size_t need = as_cache_group_bytes(B, H, S, d, P, g, cache_dt);
+  if (q_first < 0 || q_count < 1 || q_first + q_count > P)
+    return fail(AS_ERR_INVALID_ARG, "query partitions [%d, %d) outside [0, %d)", q_first, q_first + q_count, P);
+  const size_t need = as_cache_cp_bytes(B, H, S, d, P, g, cache_dt, q_count);
   if (!buf || (reinterpret_cast<uintptr_t>(buf) & 255u) != 0)
     return fail(AS_ERR_INVALID_ARG, "cache buffer must be non-null and 256-byte aligned");
   if (bytes < need) return fail(AS_ERR_INVALID_ARG, "cache buffer has %zu bytes, needs %zu", bytes, need);
@@ -321,11 +333,19 @@ as_status as_cache_group_init(as_cache* c, void* buf, size_t bytes, int B, int H
   c->g = g;
   c->n_groups = (P + g - 1) / g;
   c->cache_dt = cache_dt;
+  c->q_first = q_first;
+  c->q_count = q_count;
   c->out_planes = buf;
-  const size_t out_bytes = static_cast<size_t>(c->n_groups) * B * H * S * d * (cache_dt == AS_BF16 ? 2 : 4);
+  const size_t out_bytes =
+      static_cast<size_t>(c->n_groups) * B * H * q_count * (S / P) * d * (cache_dt == AS_BF16 ? 2 : 4);
   c->lse_planes = reinterpret_cast<float*>(static_cast<char*>(buf) + out_bytes);
   for (int x = 0; x < AS_MAX_P * AS_MAX_P; ++x) c->t_c[x] = -1;
   return ok();
+}
+
+as_status as_cache_group_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, int g,
+                              as_dtype cache_dt) {
+  return as_cache_cp_init(c, buf, bytes, B, H, S, d, P, g, cache_dt, 0, P);
 }
 
 as_status as_cache_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, as_dtype cache_dt) {
@@ -340,11 +360,23 @@ as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step, ui
   return ok();
 }
 
-// as_step and as_step_local; local_out == nullptr: no precomputed local states
+// K/V layout of a step: kv_rows rows per head in k and v, KV partition j at
+// rows [kv_slot[j] * n, (kv_slot[j] + 1) * n) (kv_slot == nullptr: slot j,
+// the whole sequence in place)
+struct KvLayout {
+  int kv_rows;
+  const int32_t* kv_slot;
+};
+
+// as_step, as_step_local and as_step_cp.  The cache's query partitions
+// [q_first, q_first + q_count) are the query rows of q, out and lse
+// (q_count * n rows per head); local_out == nullptr: no precomputed local
+// states.
 static as_status step_impl(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
                            const uint8_t* h_plan, int step, const float* local_out, const float* local_lse,
-                           float* out, float* lse, uint8_t* h_hit, int32_t* h_age, void* stream) {
-  Range nvtx_range(local_out ? "as_step_local" : "as_step");
+                           float* out, float* lse, uint8_t* h_hit, int32_t* h_age, void* stream,
+                           const KvLayout& kvl, const char* name) {
+  Range nvtx_range(name);
   as_status s = check_cache(c);
   if (s != AS_OK) return s;
   if (dt != AS_F32 && dt != AS_BF16) return fail(AS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
@@ -355,76 +387,103 @@ static as_status step_impl(as_cache* c, const void* q, const void* k, const void
     return fail(AS_ERR_INVALID_ARG, "local states must be non-null and 16-byte aligned");
   if (!(scale > 0.f)) return fail(AS_ERR_INVALID_ARG, "scale must be > 0");
   const int B = c->B, H = c->H, S = c->S, d = c->d, P = c->P, n = S / P, g = c->g, NG = c->n_groups;
+  const int i0 = c->q_first, nq = c->q_count, Sq = nq * n;
+  if (local_out && nq != P)
+    return fail(AS_ERR_UNSUPPORTED, "local states need a cache over every query partition");
   uint8_t hit[AS_MAX_P * AS_MAX_P];
   int32_t age[AS_MAX_P * AS_MAX_P];
   if ((s = resolve(c, h_plan, step, hit, age)) != AS_OK) return s;
+  // every KV partition the cache's rows compute must be in k / v
+  if (kvl.kv_slot) {
+    uint64_t used = 0;
+    for (int j = 0; j < P; ++j) {
+      bool needed = false;
+      for (int i = i0; i < i0 + nq; ++i) needed |= h_plan[i * P + j] != AS_PLAN_REUSE;
+      const int sl = kvl.kv_slot[j];
+      if (sl < 0) {
+        if (needed) return fail(AS_ERR_INVALID_ARG, "KV partition %d is computed by the plan but not in the buffer", j);
+        continue;
+      }
+      if (static_cast<long long>(sl + 1) * n > kvl.kv_rows)
+        return fail(AS_ERR_INVALID_ARG, "KV partition %d at slot %d lies beyond the buffer's %d rows", j, sl,
+                    kvl.kv_rows);
+      if (sl >= 64 || (used >> sl) & 1u) return fail(AS_ERR_INVALID_ARG, "KV slot %d given twice (or >= 64)", sl);
+      used |= uint64_t(1) << sl;
+    }
+  }
   if ((s = check_device()) != AS_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   // a plain-fresh diagonal pair whose state the caller already holds
   auto local_of = [&](int i) { return local_out != nullptr && h_plan[i * P + i] == AS_PLAN_FRESH; };
 
   // fresh pairs: composite of the plain-fresh partitions -> out/lse; the
-  // stored members of each group -> one composed state in the group's plane
+  // stored members of each group -> one composed state in the group's plane.
+  // Block b is query partition i0 + b, at local rows [b n, (b + 1) n).
   asp::AttnLaunch L;
   base_launch(L, q, k, v, B, H, S, d, P, scale);
-  L.n_blocks = P;
+  L.S = Sq;
+  L.S_kv = kvl.kv_rows;
+  for (int j = 0; j < P; ++j) L.kv_row0[j] = kvl.kv_slot ? std::max(0, kvl.kv_slot[j]) * n : j * n;
+  L.n_blocks = nq;
   L.block_rows = n;
   L.block_row0 = 0;
   bool any_fresh = false;
-  for (int i = 0; i < P; ++i) {
+  for (int b = 0; b < nq; ++b) {
+    const int i = i0 + b;
     for (int j = 0; j < P; ++j) {
       const uint8_t pc = h_plan[i * P + j];
       uint8_t kc = pc == AS_PLAN_FRESH ? AS_KCODE_COMPOSE : pc == AS_PLAN_FRESH_STORE ? AS_KCODE_EMIT : AS_KCODE_SKIP;
       if (j == i && local_of(i)) kc = AS_KCODE_SKIP;
-      L.code[i * P + j] = kc;
+      L.code[b * P + j] = kc;
       any_fresh |= kc != AS_KCODE_SKIP;
     }
   }
   for (int j = 0; j < P; ++j) L.dest_of[j] = static_cast<int8_t>(j / g);
-  // every query partition reads the same KV list: one block of S rows, so
+  // every query partition reads the same KV list: one block of all rows, so
   // query tiles are not cut at partition boundaries
   bool uniform = true;
-  for (int i = 1; i < P && uniform; ++i) uniform = std::memcmp(L.code, L.code + i * P, P) == 0;
+  for (int b = 1; b < nq && uniform; ++b) uniform = std::memcmp(L.code, L.code + b * P, P) == 0;
   if (uniform) {
     L.n_blocks = 1;
-    L.block_rows = S;
+    L.block_rows = Sq;
   }
   L.out = out;
   L.lse = lse;
-  L.out_rows = S;
+  L.out_rows = Sq;
   L.out_row0 = 0;
   L.dst_out = c->out_planes;
   L.dst_bf16 = c->cache_dt == AS_BF16;
   L.dst_lse = c->lse_planes;
-  L.dst_rows = S;
+  L.dst_rows = Sq;
   L.dst_row0 = 0;
-  L.dst_plane_out = static_cast<long long>(B) * H * S * d;
-  L.dst_plane_lse = static_cast<long long>(B) * H * S;
+  L.dst_plane_out = static_cast<long long>(B) * H * Sq * d;
+  L.dst_plane_lse = static_cast<long long>(B) * H * Sq;
   if (any_fresh && (s = launch_attn(L, dt, st)) != AS_OK) return s;
 
   // final composition: composite + local state + stored and reused group entries
   asp::ComposePlan a;
   std::memset(&a, 0, sizeof(a));
   bool need_compose = false;
-  for (int i = 0; i < P; ++i) {
+  for (int b = 0; b < nq; ++b) {
+    const int i = i0 + b;
     int cnt = 0;
     bool composite = false;
-    for (int j = 0; j < P; ++j) composite |= L.code[i * P + j] == AS_KCODE_COMPOSE;
-    if (composite) a.src[i][cnt++] = -1;
-    if (local_of(i)) a.src[i][cnt++] = -2;
+    for (int j = 0; j < P; ++j) composite |= L.code[(uniform ? 0 : b) * P + j] == AS_KCODE_COMPOSE;
+    if (composite) a.src[b][cnt++] = -1;
+    if (local_of(i)) a.src[b][cnt++] = -2;
     for (int G = 0; G < NG; ++G)
       if (group_mask(h_plan, P, g, i, G, AS_PLAN_REUSE) || group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE))
-        a.src[i][cnt++] = static_cast<int8_t>(G);
+        a.src[b][cnt++] = static_cast<int8_t>(G);
     // a row whose only source is the composite already holds its final state
-    a.nsrc[i] = (cnt == 1 && composite) ? 0 : static_cast<uint8_t>(cnt);
-    need_compose |= a.nsrc[i] > 0;
+    a.nsrc[b] = (cnt == 1 && composite) ? 0 : static_cast<uint8_t>(cnt);
+    need_compose |= a.nsrc[b] > 0;
   }
   if (need_compose) {
     a.B = B;
     a.H = H;
-    a.S = S;
+    a.S = Sq;
     a.d = d;
-    a.P = P;
+    a.P = nq;
     a.n = n;
     a.cache_out = c->out_planes;
     a.cache_bf16 = c->cache_dt == AS_BF16;
@@ -439,7 +498,7 @@ static as_status step_impl(as_cache* c, const void* q, const void* k, const void
     if (e != cudaSuccess) return cuda_fail(e, "step compose launch");
   }
 
-  for (int i = 0; i < P; ++i)
+  for (int i = i0; i < i0 + nq; ++i)
     for (int G = 0; G < NG; ++G) {
       const uint64_t m = group_mask(h_plan, P, g, i, G, AS_PLAN_FRESH_STORE);
       if (!m) continue;
@@ -454,14 +513,34 @@ static as_status step_impl(as_cache* c, const void* q, const void* k, const void
 as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
                   const uint8_t* h_plan, int step, float* out, float* lse, uint8_t* h_hit, int32_t* h_age,
                   void* stream) {
-  return step_impl(c, q, k, v, dt, scale, h_plan, step, nullptr, nullptr, out, lse, h_hit, h_age, stream);
+  as_status s = check_cache(c);
+  if (s != AS_OK) return s;
+  if (c->q_count != c->P)
+    return fail(AS_ERR_INVALID_ARG, "as_step needs a cache over every query partition; use as_step_cp");
+  return step_impl(c, q, k, v, dt, scale, h_plan, step, nullptr, nullptr, out, lse, h_hit, h_age, stream,
+                   KvLayout{c->S, nullptr}, "as_step");
 }
 
 as_status as_step_local(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
                         const uint8_t* h_plan, int step, const float* local_out, const float* local_lse, float* out,
                         float* lse, uint8_t* h_hit, int32_t* h_age, void* stream) {
   if (!local_out || !local_lse) return fail(AS_ERR_INVALID_ARG, "null local states");
-  return step_impl(c, q, k, v, dt, scale, h_plan, step, local_out, local_lse, out, lse, h_hit, h_age, stream);
+  as_status s = check_cache(c);
+  if (s != AS_OK) return s;
+  return step_impl(c, q, k, v, dt, scale, h_plan, step, local_out, local_lse, out, lse, h_hit, h_age, stream,
+                   KvLayout{c->S, nullptr}, "as_step_local");
+}
+
+as_status as_step_cp(as_cache* c, const void* q, const void* k_buf, const void* v_buf, int kv_rows,
+                     const int32_t* h_kv_slot, as_dtype dt, float scale, const uint8_t* h_plan, int step, float* out,
+                     float* lse, uint8_t* h_hit, int32_t* h_age, void* stream) {
+  as_status s = check_cache(c);
+  if (s != AS_OK) return s;
+  if (!h_kv_slot) return fail(AS_ERR_INVALID_ARG, "null KV slot map");
+  if (kv_rows < 1 || static_cast<long long>(kv_rows) * c->d >= (1ll << 31))
+    return fail(AS_ERR_INVALID_ARG, "kv_rows must be >= 1 and kv_rows * d < 2^31 (got %d)", kv_rows);
+  return step_impl(c, q, k_buf, v_buf, dt, scale, h_plan, step, nullptr, nullptr, out, lse, h_hit, h_age, stream,
+                   KvLayout{kv_rows, h_kv_slot}, "as_step_cp");
 }
 
 as_status as_device_status(void* stream, uint32_t* h_bits) {
@@ -663,6 +742,7 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
   if (c->P != P) return fail(AS_ERR_INVALID_ARG, "cache and planner disagree on P");
   if (c->g != pl->g)
     return fail(AS_ERR_INVALID_ARG, "cache groups of %d partitions, planner groups of %d", c->g, pl->g);
+  if (c->q_count != c->P) return fail(AS_ERR_UNSUPPORTED, "the planner needs a cache over every query partition");
   if (!lse_full || !local_anchor || !h_plan) return fail(AS_ERR_INVALID_ARG, "null pointer");
   if ((s = check_drift_inputs(local_anchor, local_anchor)) != AS_OK) return s;
   const int B = c->B, H = c->H, S = c->S, d = c->d, n = S / P;

@@ -365,17 +365,19 @@ struct KvSchedule {
   int group_dest[AS_MAX_P + 1];  // -1: the composite output; >= 0: destination plane
 };
 
+// KV partition j covers K/V rows [kv_row0[j], kv_row0[j] + n); partitions whose
+// rows are adjacent merge into one range.
 __device__ __forceinline__ void build_schedule(const uint8_t* code_row, const int8_t* dest_of,
-                                               int P, int n, KvSchedule& s) {
+                                               const int* kv_row0, int P, int n, KvSchedule& s) {
   s.n_ranges = 0;
   s.n_groups = 0;
   for (int j = 0; j < P; ++j) {
     if (code_row[j] != AS_KCODE_COMPOSE) continue;
-    if (s.n_ranges > 0 && s.range_hi[s.n_ranges - 1] == j * n) {
-      s.range_hi[s.n_ranges - 1] = (j + 1) * n;
+    if (s.n_ranges > 0 && s.range_hi[s.n_ranges - 1] == kv_row0[j]) {
+      s.range_hi[s.n_ranges - 1] = kv_row0[j] + n;
     } else {
-      s.range_lo[s.n_ranges] = j * n;
-      s.range_hi[s.n_ranges] = (j + 1) * n;
+      s.range_lo[s.n_ranges] = kv_row0[j];
+      s.range_hi[s.n_ranges] = kv_row0[j] + n;
       ++s.n_ranges;
     }
   }
@@ -390,18 +392,18 @@ __device__ __forceinline__ void build_schedule(const uint8_t* code_row, const in
     const int dst = dest_of[j];
     if (s.n_groups > 0 && s.group_dest[s.n_groups - 1] == dst) {
       // same destination as the previous emitted partition: one group
-      if (s.range_hi[s.n_ranges - 1] == j * n) {
-        s.range_hi[s.n_ranges - 1] = (j + 1) * n;
+      if (s.range_hi[s.n_ranges - 1] == kv_row0[j]) {
+        s.range_hi[s.n_ranges - 1] = kv_row0[j] + n;
       } else {
-        s.range_lo[s.n_ranges] = j * n;
-        s.range_hi[s.n_ranges] = (j + 1) * n;
+        s.range_lo[s.n_ranges] = kv_row0[j];
+        s.range_hi[s.n_ranges] = kv_row0[j] + n;
         ++s.n_ranges;
         ++s.group_count[s.n_groups - 1];
       }
       continue;
     }
-    s.range_lo[s.n_ranges] = j * n;
-    s.range_hi[s.n_ranges] = (j + 1) * n;
+    s.range_lo[s.n_ranges] = kv_row0[j];
+    s.range_hi[s.n_ranges] = kv_row0[j] + n;
     s.group_first[s.n_groups] = s.n_ranges;
     s.group_count[s.n_groups] = 1;
     s.group_dest[s.n_groups] = dst;

@@ -21,9 +21,14 @@ namespace asp {
 // Everything an attention launch needs, passed by value as a kernel parameter.
 struct AttnLaunch {
   const void* q;  // [B,H,S,d] (used by the SIMT path; the TMA path reads via tensor maps)
-  const void* k;
+  const void* k;  // [B,H,S_kv,d]
   const void* v;
-  int B, H, S, d, P, n;  // n = S / P
+  int B, H, S, d, P, n;  // S: query (and output) rows per head; n: rows per partition
+  // K/V rows per head, and the first K/V row of each KV partition j (its
+  // n rows are contiguous); for one GPU holding every partition S_kv = S and
+  // kv_row0[j] = j * n
+  int S_kv;
+  int kv_row0[AS_MAX_P];
   float scale;
   // query rows: n_blocks blocks of block_rows rows starting at block_row0; block b
   // uses row b of `code` ([n_blocks][P])

@@ -30,10 +30,10 @@ __global__ void __launch_bounds__(ROWS) attn_simt_kernel(const __grid_constant__
   const int q_lo = block_lo + qt * ROWS;
   const int q_hi = min(min(q_lo + ROWS, block_lo + L.block_rows), L.S);
   const float* Q = static_cast<const float*>(L.q) + static_cast<long long>(bh) * L.S * D;
-  const float* K = static_cast<const float*>(L.k) + static_cast<long long>(bh) * L.S * D;
-  const float* V = static_cast<const float*>(L.v) + static_cast<long long>(bh) * L.S * D;
+  const float* K = static_cast<const float*>(L.k) + static_cast<long long>(bh) * L.S_kv * D;
+  const float* V = static_cast<const float*>(L.v) + static_cast<long long>(bh) * L.S_kv * D;
 
-  if (threadIdx.x == 0) build_schedule(L.code + blk * L.P, L.dest_of, L.P, L.n, sched);
+  if (threadIdx.x == 0) build_schedule(L.code + blk * L.P, L.dest_of, L.kv_row0, L.P, L.n, sched);
   for (int i = threadIdx.x; i < ROWS * D; i += ROWS) {
     const int r = i / D, col = i % D;
     sQ[r * (D + 1) + col] = (q_lo + r < L.S) ? Q[static_cast<long long>(q_lo + r) * D + col] : 0.f;

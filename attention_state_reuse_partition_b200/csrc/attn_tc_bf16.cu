@@ -206,7 +206,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     mbar_init(&c.drain, 1);
     c.abort = 0;
-    build_schedule(L.code + blk * L.P, L.dest_of, L.P, L.n, c.sched);
+    build_schedule(L.code + blk * L.P, L.dest_of, L.kv_row0, L.P, L.n, c.sched);
     c.n_tiles = count_tiles(c.sched);
     mbar_fence_init();
   }
@@ -539,7 +539,7 @@ template <int D>
 cudaError_t launch_d(const AttnLaunch& L, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   const int BH = L.B * L.H;
-  if (!make_tmap(&tq, L.q, BH, L.S, D) || !make_tmap(&tk, L.k, BH, L.S, D) || !make_tmap(&tv, L.v, BH, L.S, D))
+  if (!make_tmap(&tq, L.q, BH, L.S, D) || !make_tmap(&tk, L.k, BH, L.S_kv, D) || !make_tmap(&tv, L.v, BH, L.S_kv, D))
     return cudaErrorInvalidValue;
   constexpr int smem = smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

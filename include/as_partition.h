@@ -120,6 +120,10 @@ typedef struct as_cache {
   int32_t t_c[AS_MAX_P * AS_MAX_P];
   int g, n_groups;
   uint64_t member[AS_MAX_P * AS_MAX_P];
+  /* the cache's query partitions [q_first, q_first + q_count): every one
+   * (0, P) except for one rank of a context-parallel group (as_cache_cp_init);
+   * its planes then hold q_count * S/P rows per head instead of S */
+  int q_first, q_count;
 } as_cache;
 
 /* Bytes of device memory a cache with one entry per pair (g = 1) needs.
@@ -168,9 +172,10 @@ as_status as_plan_resolve(const as_cache* c, const uint8_t* h_plan, int step,
  * entry.  h_hit / h_age (may be NULL) as in as_plan_resolve.  The plan is
  * checked before any launch: on AS_ERR_CACHE_MISS or AS_ERR_INVALID_ARG
  * nothing is launched and the cache is unchanged.  The cache must have been
- * initialised for the same B, H, S, d, P: q, k, v are read and out, lse
- * written with the cache's sizes, which the library cannot check against the
- * caller's buffers (the Python binding does).  The call neither allocates nor
+ * initialised for the same B, H, S, d, P, over every query partition
+ * (AS_ERR_INVALID_ARG otherwise; one rank's cache goes to as_step_cp): q, k,
+ * v are read and out, lse written with the cache's sizes, which the library
+ * cannot check against the caller's buffers (the Python binding does).  The call neither allocates nor
  * synchronises, so it can be captured in a CUDA graph: a replay repeats the
  * device work with the captured plan and pointers, while the host
  * bookkeeping (checks, hit/age, t_c, member) happens once, at the captured
@@ -191,6 +196,45 @@ as_status as_step(as_cache* c, const void* q, const void* k, const void* v, as_d
 as_status as_step_local(as_cache* c, const void* q, const void* k, const void* v, as_dtype dt, float scale,
                         const uint8_t* h_plan, int step, const float* local_out, const float* local_lse,
                         float* out, float* lse, uint8_t* h_hit, int32_t* h_age, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Context parallelism: one rank of a group that splits the P partitions by
+ * query partition (DiTango review page: Referee Report "Summary", group-wise
+ * KV transfer across GPUs; "Core claim", cached states stand in for far
+ * partitions, so a reused pair needs no KV transfer).  The rank owns query
+ * partitions [q_first, q_first + q_count) and their cache entries; before a
+ * step it fetches (by its own collectives) only the K/V partitions that its
+ * rows of the plan compute fresh, into a compact buffer.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of a cache for q_count query partitions (1 <= q_count <= P):
+ * n_groups * B*H*q_count*(S/P) * (d * sizeof(OUT entry) + 4).  0 for invalid
+ * sizes. */
+size_t as_cache_cp_bytes(int B, int H, int S, int d, int P, int g, as_dtype cache_dt, int q_count);
+
+/* As as_cache_group_init for the query partitions [q_first, q_first +
+ * q_count) of a sequence of S rows in P partitions: OUT planes
+ * [n_groups][B,H,q_count*S/P,d], LSE planes [n_groups][B,H,q_count*S/P],
+ * entry (i, G) at the local rows of partition i ((i - q_first) * S/P).
+ * AS_ERR_INVALID_ARG if the run leaves [0, P). */
+as_status as_cache_cp_init(as_cache* c, void* buf, size_t bytes, int B, int H, int S, int d, int P, int g,
+                           as_dtype cache_dt, int q_first, int q_count);
+
+/* as_step for the rank that owns the cache's query partitions.
+ *   q, out [B,H,q_count*S/P,d] and lse [B,H,q_count*S/P]: the rank's query
+ *   rows (partition q_first at local row 0).  k_buf, v_buf [B,H,kv_rows,d]
+ *   (dt, device, 16-byte aligned): KV partition j at rows
+ *   [h_kv_slot[j] * S/P, (h_kv_slot[j] + 1) * S/P) when h_kv_slot[j] >= 0
+ *   (host int32 [P]; -1 = not in the buffer).
+ *   h_plan is the group's [P*P] plan; only rows q_first .. q_first+q_count-1
+ *   are read beyond their codes, and h_hit / h_age are 0 in the other rows.
+ * Errors, before any launch: AS_ERR_INVALID_ARG if a pair of the rank's rows
+ * with code 1 or 2 names a KV partition that is not in the buffer, if a slot
+ * lies beyond kv_rows or is given twice; then as as_step.  The result equals
+ * as_step's rows for those partitions on the whole sequence. */
+as_status as_step_cp(as_cache* c, const void* q, const void* k_buf, const void* v_buf, int kv_rows,
+                     const int32_t* h_kv_slot, as_dtype dt, float scale, const uint8_t* h_plan, int step, float* out,
+                     float* lse, uint8_t* h_hit, int32_t* h_age, void* stream);
 
 /* Synchronise `stream`, then read and clear the device error word that the
  * kernels' bounded waits set.  *h_bits receives the raw bits (may be NULL).

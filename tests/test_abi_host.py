@@ -406,3 +406,53 @@ def test_drift_entry_points_reject_misaligned_local_states(api):
         st, msg = _status(call)
         assert st == _lib.AS_ERR_INVALID_ARG, (name, st, msg)
         assert "16-byte aligned" in msg, (name, msg)
+
+
+def test_rank_cache_and_step_cp_checks(api):
+    """One rank's cache (context parallelism) and as_step_cp's checks, all on
+    the host before any launch: a KV partition that the rank's rows compute
+    but the buffer lacks, a slot beyond the buffer or given twice, and a rank
+    cache passed to as_step are refused; misses are checked only in the
+    rank's own rows."""
+    from attention_state_reuse_partition_b200 import _lib
+    L = _lib.LIB
+    B, H, S, d, P = 1, 2, 8 * 64, 64, 8
+    n = S // P
+    assert api.as_cache_cp_bytes(B, H, S, d, P, 3) == 3 * n * B * H * (d * 4 + 4) * P
+    assert api.as_cache_cp_bytes(B, H, S, d, P, 0) == 0 and api.as_cache_cp_bytes(B, H, S, d, P, P + 1) == 0
+    with pytest.raises(api.AsError):
+        api.AsCache.host_only(B, H, S, d, P, q_first=6, q_count=3)
+    c = api.AsCache.host_only(B, H, S, d, P, q_first=3, q_count=3)
+    p = 1 << 20
+    # rows 3..5 (the rank's) compute every KV partition (window fresh, the rest
+    # fresh-and-store); every other row reuses entries nobody stored, which
+    # concerns other ranks only
+    plan = np.zeros((P, P), np.uint8)
+    for i in range(3, 6):
+        plan[i] = [1 if abs(i - j) <= 1 else 2 for j in range(P)]
+    hit, age = api.as_plan_resolve(c, plan, 0)
+    assert hit.sum() == 0 and age.sum() == 0
+    own_miss = plan.copy()
+    own_miss[4, 7] = 0
+    with pytest.raises(api.AsError) as ei:
+        api.as_plan_resolve(c, own_miss, 0)
+    assert ei.value.status == _lib.AS_ERR_CACHE_MISS and "(4, 7)" in str(ei.value)
+
+    def step_cp(slots, kv_rows):
+        arr = np.ascontiguousarray(plan.reshape(-1))
+        sl = np.ascontiguousarray(np.asarray(slots, np.int32))
+        return L.as_step_cp(ctypes.byref(c.struct), p, p, p, kv_rows, sl.ctypes.data, 1, 0.125, arr.ctypes.data,
+                            0, p, p, None, None, None)
+    for slots, kv_rows, frag in [([-1, 1, 2, 3, 4, 5, 6, 7], 8 * n, "not in the buffer"),
+                                 ([0, 1, 2, 3, 4, 5, 6, 8], 8 * n, "beyond"),
+                                 ([0, 1, 2, 3, 3, 5, 6, 7], 8 * n, "twice"),
+                                 ([0, 1, 2, 3, 4, 5, 6, 7], 7 * n, "beyond")]:
+        st, msg = _status(lambda: step_cp(slots, kv_rows))
+        assert st == _lib.AS_ERR_INVALID_ARG and frag in msg, (slots, st, msg)
+    assert (c.t_c == -1).all()
+    full = api.AsCache.host_only(B, H, S, d, P)
+    st, msg = _status(lambda: L.as_step(ctypes.byref(c.struct), p, p, p, 1, 0.125,
+                                        np.ascontiguousarray(plan.reshape(-1)).ctypes.data, 0, p, p, None, None,
+                                        None))
+    assert st == _lib.AS_ERR_INVALID_ARG and "as_step_cp" in msg
+    assert full.rows == S and c.rows == 3 * n

@@ -1,0 +1,146 @@
+"""Context parallelism on CPU with gloo (world sizes 2 and 3): every rank owns
+a contiguous run of query partitions, exchanges with the others only the KV
+partitions its plan rows compute fresh, and evaluates its own rows.
+
+Checks, per rank and step of a long-trajectory construction (anchor, then
+reuse steps with window 4 and forced-fresh pairs):
+* the received buffer holds exactly the needed partitions, each equal to the
+  global K/V rows of that partition, at the slots the layout gives;
+* the bytes received equal the exchange plan's count, and on reuse steps
+  fall below an all-gather's (reused pairs move nothing);
+* the float64 oracle run on the rank's rows with ONLY the exchanged
+  partitions present (every other KV partition zeroed) equals, bit for bit,
+  the oracle's global step on those rows: states, LSEs, hit and age.  So the
+  rank never needs a partition it did not receive.
+(DiTango review page: Referee Report "Summary", group-wise KV transfer;
+"Core claim", cached states stand in for far partitions.)"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _spec():
+    from attention_state_reuse_partition_b200 import workloads as W
+    return W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16)
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from attention_state_reuse_partition_b200 import cp
+    from attention_state_reuse_partition_b200 import workloads as W
+    from oracle import as_oracle as O
+    s = _spec()
+    n = s.n
+    layout = cp.CpLayout(s.P, world)
+    mine = layout.parts(rank)
+    rows = np.concatenate([np.arange(i * n, (i + 1) * n) for i in mine])
+    ocache = O.StateCache(s.P)
+    res = []
+    for t, qq, kk, vv in W.video_trajectory(s):
+        plan = W.plan_for_step(s, t).numpy()
+        q32, k32, v32 = (x.float() for x in (qq, kk, vv))
+        k_buf, v_buf, slots = cp.exchange_kv(k32[:, :, rows], v32[:, :, rows], plan, layout, rank, n)
+        need = cp.needed_kv(plan, mine)
+        assert [j for j in range(s.P) if slots[j] >= 0] == need
+        for j in need:
+            a = int(slots[j]) * n
+            assert torch.equal(k_buf[:, :, a:a + n], k32[:, :, j * n:(j + 1) * n])
+            assert torch.equal(v_buf[:, :, a:a + n], v32[:, :, j * n:(j + 1) * n])
+        received = (len(need) - len([j for j in need if j in mine])) * 2 * s.B * s.H * n * s.d * 4
+        # what the rank can see: its own query rows, and only the exchanged KV partitions
+        qv = torch.zeros_like(q32)
+        qv[:, :, rows] = q32[:, :, rows]
+        kv_k, kv_v = torch.zeros_like(k32), torch.zeros_like(v32)
+        for j in need:
+            a = int(slots[j]) * n
+            kv_k[:, :, j * n:(j + 1) * n] = k_buf[:, :, a:a + n]
+            kv_v[:, :, j * n:(j + 1) * n] = v_buf[:, :, a:a + n]
+        # the rank's view of the plan: the rows of other ranks' query partitions
+        # are not evaluated here, so they touch no cache entry of this rank
+        own = np.full_like(plan, O.PLAN_FRESH)
+        own[list(mine)] = plan[list(mine)]
+        out, lse, hit, age = O.step(ocache, qv.double().numpy(), kv_k.double().numpy(), kv_v.double().numpy(),
+                                    own, t, s.scale, rows=rows)
+        res.append((t, out, lse, hit[list(mine)], age[list(mine)], received))
+    q.put((rank, res))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_cp_exchange_and_rank_steps_gloo(world):
+    from attention_state_reuse_partition_b200 import cp
+    from attention_state_reuse_partition_b200 import workloads as W
+    from oracle import as_oracle as O
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        try:
+            r, res = q.get(timeout=120)
+        except Exception:  # noqa: BLE001 - a rank died: report its exit code
+            for p in procs:
+                p.join(timeout=5)
+            raise AssertionError(f"a rank did not report; exit codes {[p.exitcode for p in procs]}")
+        got[r] = res
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    s = _spec()
+    n = s.n
+    layout = cp.CpLayout(s.P, world)
+    gcache = O.StateCache(s.P)
+    for t, qq, kk, vv in W.video_trajectory(s):
+        plan = W.plan_for_step(s, t).numpy()
+        f = lambda x: x.float().double().numpy()  # noqa: E731
+        out, lse, hit, age = O.step(gcache, f(qq), f(kk), f(vv), plan, t, s.scale)
+        bytes_ = cp.exchange_bytes(plan, layout, s.B, s.H, n, s.d, 4)
+        moved = 0
+        for r in range(world):
+            mine = layout.parts(r)
+            rows = np.concatenate([np.arange(i * n, (i + 1) * n) for i in mine])
+            rt, rout, rlse, rhit, rage, received = got[r][t]
+            assert rt == t
+            assert np.array_equal(rout, out[:, :, rows]), (world, r, t)
+            assert np.array_equal(rlse, lse[:, :, rows]), (world, r, t)
+            assert np.array_equal(rhit, hit[list(mine)]) and np.array_equal(rage, age[list(mine)])
+            moved += received
+        assert moved == bytes_["moved"]
+        if t > 0:
+            assert moved < bytes_["all_gather"], (t, moved, bytes_)
+
+
+def test_layout_and_exchange_plan():
+    from attention_state_reuse_partition_b200 import cp
+    lay = cp.CpLayout(10, 3)
+    assert [list(lay.parts(r)) for r in range(3)] == [[0, 1, 2, 3], [4, 5, 6], [7, 8, 9]]
+    assert [lay.owner(j) for j in range(10)] == [0] * 4 + [1] * 3 + [2] * 3
+    with pytest.raises(ValueError):
+        cp.CpLayout(2, 3)
+    # window 1 on 6 partitions over 2 ranks: rank 0 (0-2) needs 0-3, rank 1 (3-5) needs 2-5
+    P = 6
+    plan = np.array([[1 if abs(i - j) <= 1 else 0 for j in range(P)] for i in range(P)], np.uint8)
+    lay = cp.CpLayout(P, 2)
+    assert cp.needed_kv(plan, lay.parts(0)) == [0, 1, 2, 3]
+    assert cp.exchange_plan(plan, lay) == {(1, 0): [3], (0, 1): [2]}
+    assert list(cp.kv_slots([3, 0, 2], P)) == [0, -1, 1, 2, -1, -1]
+    b = cp.exchange_bytes(plan, lay, 1, 2, 4, 8, 2)
+    assert b["moved"] == 2 * (2 * 1 * 2 * 4 * 8 * 2) and b["all_gather"] == 6 * (2 * 1 * 2 * 4 * 8 * 2)
