@@ -37,6 +37,12 @@ bf16 (round to nearest even from fp32); the LSE stays fp32.  A step composes
 what the cache holds, so at a store step the stored groups enter the final
 state with the cache's precision.
 
+Residual compression of what ranks exchange (CompactFusion, "Accelerating
+Parallel Diffusion Model Serving with Residual Compression", arXiv
+2507.17511, as its listing page gives the Abstract: compressed step-wise
+residuals with lightweight error feedback): see the last section of this
+module.
+
 Every pin of this module lives in ``tests/test_oracle.py``.
 """
 from __future__ import annotations
@@ -464,3 +470,42 @@ def planner_commit_anchor(pl, cache, lse_full, rows_of, n):
             pl.w[i, G] = float(anchor_weights(np.asarray(l)[None], lse_i)[0])
             pl.alpha[i, G] = float(scale_ratios([local, o], 0)[1])
     pl.has_anchor = True
+
+
+# ---------------------------------------------------------------------------
+# residual compression of what crosses a link (CompactFusion, arXiv
+# 2507.17511, Abstract on its listing page: transmit compressed residuals --
+# step-wise activation differences -- with lightweight error feedback against
+# error accumulation), applied to the KV partitions that ranks exchange each
+# step
+# ---------------------------------------------------------------------------
+# Readings (the page names the method, not the compressor): the residual of a
+# row is taken against the receiver's reconstruction of it, which sender and
+# receiver both track (so the compression error of a step is carried into the
+# next residual: the error feedback); a row of d values is compressed to d
+# int8 codes and one fp32 scale, s = max|r| / 127, q = round-half-even(r *
+# (127 / max|r|)) clamped to [-127, 127]; the reconstruction is rounded to
+# bf16 (the attention inputs' type) after adding q * s.  Every operation is
+# taken in float32, each product and sum rounded on its own, as the kernel
+# takes them: the codes are integers decided by floating point, so both sides
+# decide them in the same precision.
+
+def residual_apply(base, q, s):
+    """x_hat = bf16(base + q * s) for rows of d values: base [..., d] (bf16
+    values), q [..., d] int8, s [...] float32."""
+    prod = (np.asarray(q).astype(np.float32) * np.asarray(s, dtype=np.float32)[..., None]).astype(np.float32)
+    tot = (np.asarray(base, dtype=np.float32) + prod).astype(np.float32)
+    return round_bf16(tot)
+
+
+def residual_encode(x, base):
+    """Compress the rows of x [..., d] against the reconstruction `base`
+    (both bf16 values): returns (q int8 [..., d], s float32 [...], the new
+    reconstruction residual_apply(base, q, s))."""
+    r = (np.asarray(x, dtype=np.float32) - np.asarray(base, dtype=np.float32)).astype(np.float32)
+    amax = np.max(np.abs(r), axis=-1).astype(np.float32)
+    nz = amax > 0
+    inv = np.where(nz, np.float32(127.0) / np.where(nz, amax, np.float32(1.0)), np.float32(0.0)).astype(np.float32)
+    q = np.clip(np.rint((r * inv[..., None]).astype(np.float32)), -127, 127).astype(np.int8)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    return q, s, residual_apply(base, q, s)

@@ -585,6 +585,82 @@ def pin_planner_trajectory_grouped(o):
     _close(out1, _sdpa(q, k, v, 0.5), TOL, "grouped planner reuse of unchanged states")
 
 
+# ---------------------------------------------------------------------------
+# residual compression pins (CompactFusion, arXiv 2507.17511, Abstract on its
+# listing page: compressed step-wise residuals with error feedback; the
+# compressor read as int8 codes with one fp32 scale per row)
+# ---------------------------------------------------------------------------
+
+def _bf16_values(r, shape, scale=1.0):
+    return as_oracle.round_bf16(r.normal(size=shape) * scale)
+
+
+def pin_residual_exact(o):
+    """A residual that is k * 2^-6 with integer |k| <= 127 and 127 reached in
+    every row is coded exactly: q = k, s = 2^-6, and the reconstruction is
+    the input (k * 2^-6 needs 7 significant bits, which bf16 holds)."""
+    r = _rng(50)
+    k = r.integers(-127, 128, size=(5, 64))
+    k[:, 3] = 127
+    k[1, 3] = -127
+    x = k * 2.0 ** -6
+    q, s, xh = o.residual_encode(x, np.zeros_like(x))
+    assert np.array_equal(q.astype(np.int64), k)
+    assert np.all(s == np.float32(2.0 ** -6))
+    assert np.array_equal(xh, x)
+
+
+def pin_residual_bound(o):
+    """|x - x_hat| <= s / 2 (the quantisation step, half of it) plus the bf16
+    rounding of the reconstruction (2^-8 relative); |q| <= 127 with the
+    largest residual of every row coded as +-127; s = max|r| / 127; the
+    reconstruction holds bf16 values."""
+    r = _rng(51)
+    for d in (64, 128):
+        x = _bf16_values(r, (7, 3, d))
+        base = _bf16_values(r, (7, 3, d), 0.9)
+        q, s, xh = o.residual_encode(x, base)
+        res = x - base
+        amax = np.max(np.abs(res), axis=-1)
+        _close(s, amax / 127.0, 1e-6 * float(amax.max()), "scale")
+        assert np.all(np.abs(q.astype(np.int64)) <= 127)
+        assert np.all(np.max(np.abs(q.astype(np.int64)), axis=-1) == 127)
+        err = np.abs(x - xh)
+        assert np.all(err <= s[..., None] * 0.5 * (1 + 1e-5) + 2.0 ** -8 * np.abs(xh) + 1e-30), float(err.max())
+        assert np.array_equal(as_oracle.round_bf16(xh), xh)
+
+
+def pin_residual_zero(o):
+    r = _rng(52)
+    x = _bf16_values(r, (4, 64))
+    q, s, xh = o.residual_encode(x, x)
+    assert not q.any() and not s.any() and np.array_equal(xh, x)
+
+
+def pin_residual_error_feedback(o):
+    """The page's point of error feedback: coding each step's residual against
+    the reconstruction keeps the error of every step within that step's own
+    bound over a 32-step random walk, while coding the difference of the true
+    consecutive values and accumulating the decoded differences drifts
+    beyond it."""
+    r = _rng(53)
+    x = _bf16_values(r, (16, 64))
+    rec = x.copy()                       # both sides start from one exact send
+    acc = x.copy()                       # no feedback: decoded differences accumulated
+    prev = x.copy()
+    drift = 0.0
+    for t in range(32):
+        x = as_oracle.round_bf16(x + 0.05 * r.normal(size=x.shape))
+        q, s, rec = o.residual_encode(x, rec)
+        bound = s[..., None] * 0.5 * (1 + 1e-5) + 2.0 ** -8 * np.abs(rec)
+        assert np.all(np.abs(x - rec) <= bound + 1e-30), t
+        qd, sd, _ = o.residual_encode(x, prev)
+        acc = as_oracle.round_bf16(acc + qd.astype(np.float64) * sd[..., None])
+        prev = x
+        drift = max(drift, float(np.max(np.abs(x - acc) - bound)))
+    assert drift > 0, "without feedback the error should leave the per-step bound"
+
+
 PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_forms,
         pin_compose_closed, pin_assoc_comm, pin_split_invariance, pin_single_partition,
         pin_plan_golden, pin_step_all_fresh, pin_step_reuse_identical, pin_step_reuse_mixed,
@@ -592,7 +668,8 @@ PINS = [pin_bruteforce_loops, pin_torch_sdpa_full, pin_scipy_lse, pin_closed_for
         pin_round_bf16, pin_plan_grouped_golden, pin_step_grouped_identical, pin_step_grouped_mixed,
         pin_step_bf16_cache,
         pin_planner_group_weights, pin_planner_select_grouped, pin_planner_trajectory_grouped,
-        pin_planner_commit_closed_form]
+        pin_planner_commit_closed_form,
+        pin_residual_exact, pin_residual_bound, pin_residual_zero, pin_residual_error_feedback]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -607,7 +684,7 @@ def test_oracle_passes_pin(pin):
 _orig = {name: getattr(as_oracle, name) for name in
          ("attention_state", "compose", "compose_pair", "resolve_plan", "step", "partition_bounds",
           "anchor_weights", "scale_ratios", "local_drift", "select_plan", "ase", "round_bf16", "n_groups",
-          "planner_commit_anchor")}
+          "planner_commit_anchor", "residual_encode", "residual_apply")}
 
 
 def _m_no_normalise(q, k, v, scale):
@@ -751,6 +828,29 @@ def _m_ase_no_alpha(w, alpha, drift):
     return _orig["ase"](w, np.ones_like(np.asarray(alpha, dtype=np.float64)), drift)
 
 
+def _m_residual_scale_255(x, base):
+    r = (np.asarray(x, np.float32) - np.asarray(base, np.float32)).astype(np.float32)
+    amax = np.max(np.abs(r), axis=-1).astype(np.float32)
+    inv = np.where(amax > 0, np.float32(255.0) / np.where(amax > 0, amax, 1), 0).astype(np.float32)
+    q = np.clip(np.rint(r * inv[..., None]), -127, 127).astype(np.int8)
+    s = (amax / np.float32(255.0)).astype(np.float32)
+    return q, s, as_oracle.residual_apply(base, q, s)
+
+
+def _m_residual_truncate(x, base):
+    r = (np.asarray(x, np.float32) - np.asarray(base, np.float32)).astype(np.float32)
+    amax = np.max(np.abs(r), axis=-1).astype(np.float32)
+    inv = np.where(amax > 0, np.float32(127.0) / np.where(amax > 0, amax, 1), 0).astype(np.float32)
+    q = np.clip(np.trunc(r * inv[..., None]), -127, 127).astype(np.int8)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    return q, s, as_oracle.residual_apply(base, q, s)
+
+
+def _m_residual_no_bf16(base, q, s):
+    prod = (np.asarray(q).astype(np.float32) * np.asarray(s, np.float32)[..., None]).astype(np.float32)
+    return (np.asarray(base, np.float32) + prod).astype(np.float64)
+
+
 def _m_commit_alpha_inverted(pl, cache, lse_full, rows_of, n):
     _orig["planner_commit_anchor"](pl, cache, lse_full, rows_of, n)
     pl.alpha = np.where(pl.alpha > 0, 1.0 / np.where(pl.alpha > 0, pl.alpha, 1.0), 0.0)
@@ -783,6 +883,9 @@ MUTANTS = {
     "n_groups: drops the short last group": ("n_groups", _m_groups_floor),
     "select_plan: a reused group takes its window members too": ("select_plan", _m_select_group_window),
     "planner_commit_anchor: inverted scale ratio": ("planner_commit_anchor", _m_commit_alpha_inverted),
+    "residual_encode: scale max/255": ("residual_encode", _m_residual_scale_255),
+    "residual_encode: codes truncated": ("residual_encode", _m_residual_truncate),
+    "residual_apply: reconstruction not rounded to bf16": ("residual_apply", _m_residual_no_bf16),
 }
 
 
