@@ -25,7 +25,8 @@ EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as
            "as_debug_exp2", "as_planner_init", "as_planner_scratch_bytes", "as_local_states", "as_plan_drift",
            "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static",
            "as_cache_group_bytes", "as_cache_group_init", "as_planner_group_init", "as_plan_select_grouped",
-           "as_step_local", "as_cache_cp_bytes", "as_cache_cp_init", "as_step_cp")
+           "as_step_local", "as_cache_cp_bytes", "as_cache_cp_init", "as_step_cp", "as_residual_encode",
+           "as_residual_decode")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -100,6 +101,10 @@ def _load() -> ctypes.CDLL:
     lib.as_cache_cp_init.restype = c_int
     lib.as_cache_cp_init.argtypes = [ctypes.POINTER(AsCacheStruct), vp, sz, c_int, c_int, c_int, c_int, c_int,
                                      c_int, c_int, c_int, c_int]
+    lib.as_residual_encode.restype = c_int
+    lib.as_residual_encode.argtypes = [vp, vp, vp, vp, ctypes.c_int64, c_int, vp]
+    lib.as_residual_decode.restype = c_int
+    lib.as_residual_decode.argtypes = [vp, vp, vp, ctypes.c_int64, c_int, vp]
     lib.as_step_cp.restype = c_int
     lib.as_step_cp.argtypes = [ctypes.POINTER(AsCacheStruct), vp, vp, vp, c_int, vp, c_int, c_float, vp, c_int,
                                vp, vp, vp, vp, vp]

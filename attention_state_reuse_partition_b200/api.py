@@ -17,7 +17,8 @@ from ._lib import (AS_BF16, AS_F32, AS_PLAN_FRESH, AS_PLAN_FRESH_STORE, AS_PLAN_
 __all__ = ["as_partition_attn", "as_compose", "as_cache_bytes", "as_cache_init", "as_plan_resolve", "as_step",
            "as_device_status", "as_debug_timeout_probe", "as_version", "AsCache", "AsError",
            "AS_PLAN_REUSE", "AS_PLAN_FRESH", "AS_PLAN_FRESH_STORE", "AsPlanner", "as_planner_init",
-           "as_planner_scratch_bytes", "as_local_states", "as_plan_drift", "as_plan_select", "as_planner_next",
+           "as_planner_scratch_bytes", "as_local_states", "as_plan_drift", "as_plan_select", "as_planner_next", "as_residual_encode",
+           "as_residual_decode",
            "as_planner_commit_anchor", "as_plan_drift_static", "as_step_local", "as_cache_cp_bytes", "as_step_cp"]
 
 
@@ -319,6 +320,42 @@ def as_step_cp(cache: AsCache, q, k_buf, v_buf, kv_slots, plan, step: int, scale
                          int(step), _dev(out, "out"), _dev(lse, "lse"), hit.ctypes.data, age.ctypes.data,
                          _stream_ptr(stream)))
     return out, lse, hit.reshape(P, P), age.reshape(P, P)
+
+
+def _rows_d(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16 or t.dim() < 2:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, f"{name} must be bfloat16 [..., d], got {t.dtype} {tuple(t.shape)}")
+    return t.numel() // t.shape[-1], t.shape[-1]
+
+
+def as_residual_encode(x, base, codes=None, scales=None, stream=None):
+    """Residual-code the rows of x [..., d] (bf16) against the reconstruction
+    `base` (same shape, bf16), which moves to the new reconstruction in
+    place.  Returns (codes int8 [..., d], scales fp32 [...])."""
+    rows, d = _rows_d(x, "x")
+    if base.shape != x.shape or base.dtype != x.dtype:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, "base must match x in shape and dtype")
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    if codes.shape != x.shape or codes.dtype != torch.int8 or scales.shape != x.shape[:-1] \
+            or scales.dtype != torch.float32:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, "codes must be int8 like x, scales float32 [...]")
+    check(LIB.as_residual_encode(_dev(x, "x"), _dev(base, "base"), _dev(codes, "codes"), _dev(scales, "scales"),
+                                 rows, d, _stream_ptr(stream)))
+    return codes, scales
+
+
+def as_residual_decode(codes, scales, base, stream=None):
+    """The receiver's half: base <- bf16(base + codes * scales), in place."""
+    rows, d = _rows_d(base, "base")
+    if codes.shape != base.shape or codes.dtype != torch.int8 or scales.shape != base.shape[:-1] \
+            or scales.dtype != torch.float32:
+        raise AsError(_lib.AS_ERR_INVALID_ARG, "codes must be int8 like base, scales float32 [...]")
+    check(LIB.as_residual_decode(_dev(codes, "codes"), _dev(scales, "scales"), _dev(base, "base"), rows, d,
+                                 _stream_ptr(stream)))
+    return base
 
 
 def as_planner_scratch_bytes(B: int, H: int, P: int) -> int:

@@ -144,3 +144,106 @@ def gather_kv_local(k: torch.Tensor, v: torch.Tensor, needed: Sequence[int], n: 
     process (for a single-GPU stand-in of one rank)."""
     js = sorted(needed)
     return _rows(k, js, 0, n), _rows(v, js, 0, n), kv_slots(js, k.shape[2] // n)
+
+
+class CudaCodec:
+    """The library's residual codec (as_residual_encode / as_residual_decode)."""
+
+    def encode(self, x, base):
+        from attention_state_reuse_partition_b200 import api
+        return api.as_residual_encode(x, base)
+
+    def decode(self, codes, scales, base):
+        from attention_state_reuse_partition_b200 import api
+        api.as_residual_decode(codes, scales, base)
+
+
+class ResidualExchange:
+    """exchange_kv with CompactFusion's residual compression on the link
+    ("Accelerating Parallel Diffusion Model Serving with Residual
+    Compression", arXiv 2507.17511, Abstract on its listing page: transmit
+    compressed step-wise residuals, with error feedback).
+
+    The first time a rank sends KV partition j to a receiver it sends the
+    rows as they are, and both keep them as the receiver's reconstruction.
+    Later sends carry the residual against that reconstruction, coded per
+    row (d int8 codes and an fp32 scale), and both sides move the
+    reconstruction by the same coded residual (as_residual_encode on the
+    sender, as_residual_decode on the receiver), so they stay bit-identical
+    and a step's coding error is fed into the next residual.  The receiver
+    attends to its reconstruction.  State: per (receiver, partition) on the
+    sender and per partition on the receiver, [B, H, n, d] for K and for V.
+
+    `codec` provides encode(x, base) -> (codes, scales) (moving base) and
+    decode(codes, scales, base); the library's kernels by default."""
+
+    def __init__(self, layout: CpLayout, rank: int, n: int, codec=None):
+        self.layout, self.rank, self.n = layout, rank, n
+        self.codec = codec if codec is not None else CudaCodec()
+        self.send_base = {}   # (dst, j) -> (k, v): the receiver's reconstruction, as this sender tracks it
+        self.recv_base = {}   # j -> (k, v): this receiver's reconstruction of a remote partition
+        self.sent_bytes = 0   # bytes this rank sent in the last exchange
+
+    def exchange(self, k_local: torch.Tensor, v_local: torch.Tensor, plan, group=None):
+        """As exchange_kv; returns (k_buf, v_buf, slots), remote partitions as
+        reconstructed."""
+        import torch.distributed as dist
+        lay, rank, n = self.layout, self.rank, self.n
+        mine = lay.parts(rank)
+        need = needed_kv(plan, mine)
+        slots = kv_slots(need, lay.P)
+        B, H, _, d = k_local.shape
+        k_buf = torch.empty((B, H, n * len(need), d), dtype=k_local.dtype, device=k_local.device)
+        v_buf = torch.empty_like(k_buf)
+        for j in need:
+            if j in mine:
+                s = int(slots[j])
+                k_buf[:, :, s * n:(s + 1) * n] = k_local[:, :, (j - mine.start) * n:(j - mine.start + 1) * n]
+                v_buf[:, :, s * n:(s + 1) * n] = v_local[:, :, (j - mine.start) * n:(j - mine.start + 1) * n]
+        ops, post = [], []
+        sent = 0
+        for (src, dst), js in sorted(exchange_plan(plan, lay).items()):
+            if src == rank:
+                for j in js:
+                    rows = [_rows(t, [j], mine.start, n) for t in (k_local, v_local)]
+                    key = (dst, j)
+                    if key not in self.send_base:
+                        self.send_base[key] = tuple(x.clone() for x in rows)
+                        payload = rows
+                    else:
+                        payload = []
+                        for x, base in zip(rows, self.send_base[key]):
+                            payload.extend(self.codec.encode(x, base))
+                    for p in payload:
+                        ops.append(dist.P2POp(dist.isend, p, dst, group=group))
+                        sent += p.numel() * p.element_size()
+            elif dst == rank:
+                for j in js:
+                    shape = (B, H, n, d)
+                    if j not in self.recv_base:
+                        bufs = [torch.empty(shape, dtype=k_local.dtype, device=k_local.device) for _ in range(2)]
+                        post.append((j, "raw", bufs))
+                    else:
+                        bufs = []
+                        for _ in range(2):
+                            bufs.append(torch.empty(shape, dtype=torch.int8, device=k_local.device))
+                            bufs.append(torch.empty(shape[:-1], dtype=torch.float32, device=k_local.device))
+                        post.append((j, "coded", bufs))
+                    for b in bufs:
+                        ops.append(dist.P2POp(dist.irecv, b, src, group=group))
+        if ops:
+            for req in dist.batch_isend_irecv(ops):
+                req.wait()
+        for j, kind, bufs in post:
+            if kind == "raw":
+                self.recv_base[j] = (bufs[0], bufs[1])
+            else:
+                kb, vb = self.recv_base[j]
+                self.codec.decode(bufs[0], bufs[1], kb)
+                self.codec.decode(bufs[2], bufs[3], vb)
+            kb, vb = self.recv_base[j]
+            s = int(slots[j])
+            k_buf[:, :, s * n:(s + 1) * n] = kb
+            v_buf[:, :, s * n:(s + 1) * n] = vb
+        self.sent_bytes = sent
+        return k_buf, v_buf, slots

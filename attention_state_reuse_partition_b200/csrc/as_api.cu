@@ -782,6 +782,38 @@ as_status as_planner_commit_anchor(as_planner* pl, const as_cache* c, const floa
   return ok();
 }
 
+as_status as_residual_encode(const void* x, void* base, int8_t* codes, float* scales, int64_t rows, int d,
+                             void* stream) {
+  Range nvtx_range("as_residual_encode");
+  if (d != 64 && d != 128) return fail(AS_ERR_INVALID_ARG, "d must be 64 or 128 (got %d)", d);
+  if (rows < 0) return fail(AS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (rows == 0) return ok();
+  if (!x || !base || !codes || !scales) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(base) || !aligned16(codes) || !aligned16(scales))
+    return fail(AS_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  as_status s = check_device();
+  if (s != AS_OK) return s;
+  cudaError_t e = asp::launch_residual_encode(x, base, codes, scales, rows, d, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "residual encode launch");
+  return ok();
+}
+
+as_status as_residual_decode(const int8_t* codes, const float* scales, void* base, int64_t rows, int d,
+                             void* stream) {
+  Range nvtx_range("as_residual_decode");
+  if (d != 64 && d != 128) return fail(AS_ERR_INVALID_ARG, "d must be 64 or 128 (got %d)", d);
+  if (rows < 0) return fail(AS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (rows == 0) return ok();
+  if (!codes || !scales || !base) return fail(AS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(base))
+    return fail(AS_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  as_status s = check_device();
+  if (s != AS_OK) return s;
+  cudaError_t e = asp::launch_residual_decode(codes, scales, base, rows, d, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "residual decode launch");
+  return ok();
+}
+
 as_status as_debug_exp2(const float* x, float* y, int64_t n, int mode, void* stream) {
   if (n < 0 || (mode != 0 && mode != 1) || (n > 0 && (!x || !y)))
     return fail(AS_ERR_INVALID_ARG, "as_debug_exp2: bad arguments");

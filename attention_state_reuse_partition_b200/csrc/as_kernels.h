@@ -95,6 +95,12 @@ cudaError_t launch_anchor_stats(const void* cache_out, bool out_bf16, const floa
 cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st);
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st);
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st);
+// residual compression of exchanged rows [rows, d] (bf16 values, int8 codes,
+// fp32 scales); base is updated in place to the new reconstruction
+cudaError_t launch_residual_encode(const void* x, void* base, int8_t* codes, float* scales, long long rows, int d,
+                                   cudaStream_t st);
+cudaError_t launch_residual_decode(const int8_t* codes, const float* scales, void* base, long long rows, int d,
+                                   cudaStream_t st);
 cudaError_t launch_timeout_probe(unsigned int polls, unsigned int ns, cudaStream_t st);
 cudaError_t launch_exp2_probe(const float* x, float* y, long long n, int mode, cudaStream_t st);
 cudaError_t read_and_clear_dev_error(unsigned int* bits, cudaStream_t st);

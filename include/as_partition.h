@@ -236,6 +236,34 @@ as_status as_step_cp(as_cache* c, const void* q, const void* k_buf, const void* 
                      const int32_t* h_kv_slot, as_dtype dt, float scale, const uint8_t* h_plan, int step, float* out,
                      float* lse, uint8_t* h_hit, int32_t* h_age, void* stream);
 
+/* Residual compression of what a rank sends (CompactFusion, "Accelerating
+ * Parallel Diffusion Model Serving with Residual Compression", arXiv
+ * 2507.17511, Abstract on its listing page: transmit compressed step-wise
+ * residuals, with lightweight error feedback against error accumulation).
+ * Applied to the KV partitions of the context-parallel exchange (cp.py):
+ * sender and receiver each keep the receiver's reconstruction `base` of a
+ * partition's rows, and from the second send on only the coded residual
+ * crosses the link: d int8 codes and one fp32 scale per row instead of d
+ * bf16 values (132 against 256 bytes at d = 128).
+ *   Per row of d values (x, base: bf16; all float32 arithmetic, each product
+ *   and sum rounded on its own): r = x - base, s = max|r| / 127,
+ *   q = round-half-even(r * (127 / max|r|)) clamped to [-127, 127] (q = 0,
+ *   s = 0 for a zero residual), base <- bf16(base + q * s) (round to
+ *   nearest even).  Because the residual is taken against the reconstruction,
+ *   a step's coding error enters the next step's residual: the error
+ *   feedback; |x - base| <= s/2 plus the bf16 rounding after every step.
+ * x, base [rows, d] bf16; codes [rows, d] int8; scales [rows] fp32; all
+ * device, 16-byte aligned; d in {64, 128}.  Stream-ordered, no allocation.
+ * AS_ERR_INVALID_ARG for other d, negative rows, null or misaligned
+ * pointers (rows = 0 is a no-op). */
+as_status as_residual_encode(const void* x, void* base, int8_t* codes, float* scales, int64_t rows, int d,
+                             void* stream);
+
+/* The receiver's half: base <- bf16(base + q * s) for every row, exactly as
+ * as_residual_encode moved the sender's copy.  Same arguments and errors. */
+as_status as_residual_decode(const int8_t* codes, const float* scales, void* base, int64_t rows, int d,
+                             void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word that the
  * kernels' bounded waits set.  *h_bits receives the raw bits (may be NULL).
  * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, else AS_OK.

@@ -456,3 +456,18 @@ def test_rank_cache_and_step_cp_checks(api):
                                         None))
     assert st == _lib.AS_ERR_INVALID_ARG and "as_step_cp" in msg
     assert full.rows == S and c.rows == 3 * n
+
+
+def test_residual_codec_checks(api):
+    """as_residual_encode / decode refuse bad sizes and pointers on the host;
+    zero rows is a no-op even without a GPU."""
+    from attention_state_reuse_partition_b200 import _lib
+    L = _lib.LIB
+    p = 1 << 20
+    assert L.as_residual_encode(p, p, p, p, 0, 128, None) == _lib.AS_OK
+    for args, frag in [((p, p, p, p, 10, 96, None), "d must be"), ((p, p, p, p, -1, 128, None), "rows"),
+                       ((p, 0, p, p, 10, 128, None), "null"), ((p + 8, p, p, p, 10, 128, None), "aligned")]:
+        st, msg = _status(lambda: L.as_residual_encode(*args))
+        assert st == _lib.AS_ERR_INVALID_ARG and frag in msg, (args, msg)
+    st, msg = _status(lambda: L.as_residual_decode(p, p, p + 4, 10, 64, None))
+    assert st == _lib.AS_ERR_INVALID_ARG and "aligned" in msg
