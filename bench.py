@@ -21,6 +21,8 @@ Also reported on the same line (same run), in fields of the contract:
   ``roofline.partition_boundary`` the flux_image step with one state emitted
   per KV partition (ragged 576-token partitions inside the timed region);
   ``roofline.locality`` the MSE of dropping a near against a far partition;
+  ``roofline.residual_codec`` the residual codec of the context-parallel
+  exchange against the measured HBM copy bandwidth;
 * ``cpu_baseline``: the float64 oracle on the host cores -- the whole
   flux_image step, and in ``cpu_baseline.legs`` the compose-bound workload and
   the video workloads on bounded samples of rows and heads (full-step times
@@ -612,6 +614,53 @@ def run_boundary(args, device, merged_tflops: float):
             "extra_bytes_written": (s.P - 1) * s.B * s.H * s.S * (s.d + 1) * 4}
 
 
+def run_residual(args, device, peaks):
+    """The residual codec of the context-parallel exchange on what one rank
+    of video_long sends a neighbour per step at 2 ranks (4 partitions of
+    K and V: 8 x 81,920 rows of d = 128), against the measured HBM copy
+    bandwidth.  Algorithmic bytes per row: encode reads x and base and
+    writes codes, scale and base (7 d + 4); decode reads codes, scale and
+    base and writes base (5 d + 4).  Link bytes per row: d + 4 coded
+    against 2 d raw."""
+    from attention_state_reuse_partition_b200 import api
+    s = W.spec("video_long")
+    rows = 8 * s.B * s.H * s.n
+    g = torch.Generator(device=device).manual_seed(91)
+    x = torch.randn((rows, s.d), generator=g, device=device).to(torch.bfloat16)
+    base = (x.float() + 0.05 * torch.randn((rows, s.d), generator=g, device=device)).to(torch.bfloat16)
+    recv = base.clone()
+    codes = torch.empty((rows, s.d), dtype=torch.int8, device=device)
+    scales = torch.empty((rows,), dtype=torch.float32, device=device)
+    enc_base = base.clone()
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    # the kernels' work does not depend on the values (the base moves
+    # towards x from one repetition to the next)
+    ms_enc = timed(lambda: api.as_residual_encode(x, enc_base, codes, scales))
+    ms_dec = timed(lambda: api.as_residual_decode(codes, scales, recv))
+    d = s.d
+    enc_b, dec_b = rows * (7 * d + 4), rows * (5 * d + 4)
+    del x, base, recv, codes, scales, enc_base
+    torch.cuda.empty_cache()
+    return {"bound": "hbm", "workload": f"{rows} rows of d = {d} (4 video_long partitions of K and V)",
+            "encode_ms": round(ms_enc, 4), "encode_gbs": round(enc_b / (ms_enc * 1e-3) / 1e9, 1),
+            "encode_frac": round(enc_b / (ms_enc * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "decode_ms": round(ms_dec, 4), "decode_gbs": round(dec_b / (ms_dec * 1e-3) / 1e9, 1),
+            "decode_frac": round(dec_b / (ms_dec * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "peak": peaks["hbm_gbs"], "link_bytes_per_row": {"coded": d + 4, "raw": 2 * d},
+            "link_ratio": round((d + 4) / (2 * d), 4)}
+
+
 def run_video_long(args, device, g=1, cache_dtype="f32", peaks=None, with_oracle=False):
     """Long video trajectory: an anchor step, then three reuse steps (window 4,
     a seeded 10% of reused pairs forced fresh and stored each step).  With
@@ -719,7 +768,7 @@ def main():
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
     ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner",
-                                       "planner_grouped", "boundary", "locality"], default=None,
+                                       "planner_grouped", "boundary", "locality", "residual"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
@@ -758,6 +807,7 @@ def main():
               "planner": run_planner,
               "planner_grouped": lambda a, dev: run_planner(a, dev, g=4, cache_dtype="bf16"),
               "boundary": lambda a, dev: run_boundary(a, dev, float("nan")),
+              "residual": lambda a, dev: run_residual(a, dev, peaks),
               "locality": run_locality}[args.only]
         print(json.dumps({"only": args.only, **fn(args, device)}))
         return
@@ -800,6 +850,7 @@ def main():
         steps["planner_g4_bf16"] = run_planner(args, device, g=4, cache_dtype="bf16")
         roofline["steps"] = steps
         roofline["partition_boundary"] = run_boundary(args, device, achieved)
+        roofline["residual_codec"] = run_residual(args, device, peaks)
         roofline["locality"] = run_locality(args, device)
     if cpu is not None and legs:
         cpu["legs"] = {k: v for k, v in legs.items() if v is not None}
