@@ -7,16 +7,19 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libasp.so")
+# ASP_DEBUG=1 selects the checked build (device-side index checks)
+CHECKED = os.environ.get("ASP_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(PKG, "libasp_debug.so" if CHECKED else "libasp.so")
 
 AS_MAX_P = 64
-AS_OK, AS_ERR_INVALID_ARG, AS_ERR_UNSUPPORTED, AS_ERR_CACHE_MISS, AS_ERR_CUDA, AS_ERR_TIMEOUT = range(6)
+AS_OK, AS_ERR_INVALID_ARG, AS_ERR_UNSUPPORTED, AS_ERR_CACHE_MISS, AS_ERR_CUDA, AS_ERR_TIMEOUT, AS_ERR_BOUNDS = range(7)
 AS_F32, AS_BF16 = 0, 1
 AS_PLAN_REUSE, AS_PLAN_FRESH, AS_PLAN_FRESH_STORE = 0, 1, 2
 
 STATUS_NAMES = {
     AS_OK: "AS_OK", AS_ERR_INVALID_ARG: "AS_ERR_INVALID_ARG", AS_ERR_UNSUPPORTED: "AS_ERR_UNSUPPORTED",
     AS_ERR_CACHE_MISS: "AS_ERR_CACHE_MISS", AS_ERR_CUDA: "AS_ERR_CUDA", AS_ERR_TIMEOUT: "AS_ERR_TIMEOUT",
+    AS_ERR_BOUNDS: "AS_ERR_BOUNDS",
 }
 
 # every entry point declared in include/as_partition.h
@@ -26,7 +29,7 @@ EXPORTS = ("as_last_error", "as_version", "as_partition_attn", "as_compose", "as
            "as_plan_select", "as_planner_next", "as_planner_commit_anchor", "as_plan_drift_static",
            "as_cache_group_bytes", "as_cache_group_init", "as_planner_group_init", "as_plan_select_grouped",
            "as_step_local", "as_cache_cp_bytes", "as_cache_cp_init", "as_step_cp", "as_residual_encode",
-           "as_residual_decode")
+           "as_residual_decode", "as_debug_bounds_probe")
 
 
 class AsCacheStruct(ctypes.Structure):
@@ -101,6 +104,8 @@ def _load() -> ctypes.CDLL:
     lib.as_cache_cp_init.restype = c_int
     lib.as_cache_cp_init.argtypes = [ctypes.POINTER(AsCacheStruct), vp, sz, c_int, c_int, c_int, c_int, c_int,
                                      c_int, c_int, c_int, c_int]
+    lib.as_debug_bounds_probe.restype = c_int
+    lib.as_debug_bounds_probe.argtypes = [vp, ctypes.c_int64, vp]
     lib.as_residual_encode.restype = c_int
     lib.as_residual_encode.argtypes = [vp, vp, vp, vp, ctypes.c_int64, c_int, vp]
     lib.as_residual_decode.restype = c_int

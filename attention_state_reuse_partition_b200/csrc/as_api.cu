@@ -21,6 +21,12 @@
 
 namespace {
 
+#ifdef ASP_DEBUG
+constexpr bool ASP_CHECKED_BUILD = ASP_DEBUG != 0;
+#else
+constexpr bool ASP_CHECKED_BUILD = false;
+#endif
+
 constexpr uint32_t CACHE_MAGIC = 0x41535043u;    // "ASPC"
 constexpr uint32_t PLANNER_MAGIC = 0x41535050u;  // "ASPP"
 thread_local std::string g_err;
@@ -220,7 +226,10 @@ extern "C" {
 
 const char* as_last_error(void) { return g_err.c_str(); }
 
-const char* as_version(void) { return "attention-state-reuse-partition b200 0.1 (sm_100a)"; }
+const char* as_version(void) {
+  return ASP_CHECKED_BUILD ? "attention-state-reuse-partition b200 0.2 (sm_100a, checked)"
+                           : "attention-state-reuse-partition b200 0.2 (sm_100a)";
+}
 
 as_status as_partition_attn(const void* q, const void* k, const void* v, as_dtype dt, int B, int H, int S, int d,
                             int P, float scale, int q_part, const int32_t* h_kv_parts, int n_kv_parts, int compose,
@@ -260,6 +269,7 @@ as_status as_partition_attn(const void* q, const void* k, const void* v, as_dtyp
   L.dst_row0 = L.block_row0;
   L.dst_plane_out = static_cast<long long>(B) * H * R * d;
   L.dst_plane_lse = static_cast<long long>(B) * H * R;
+  L.dst_planes = compose ? 1 : n_kv_parts;
   if ((s = check_device()) != AS_OK) return s;
   if ((s = launch_attn(L, dt, static_cast<cudaStream_t>(stream))) != AS_OK) return s;
   return ok();
@@ -458,6 +468,7 @@ static as_status step_impl(as_cache* c, const void* q, const void* k, const void
   L.dst_row0 = 0;
   L.dst_plane_out = static_cast<long long>(B) * H * Sq * d;
   L.dst_plane_lse = static_cast<long long>(B) * H * Sq;
+  L.dst_planes = NG;
   if (any_fresh && (s = launch_attn(L, dt, st)) != AS_OK) return s;
 
   // final composition: composite + local state + stored and reused group entries
@@ -487,6 +498,7 @@ static as_status step_impl(as_cache* c, const void* q, const void* k, const void
     a.n = n;
     a.cache_out = c->out_planes;
     a.cache_bf16 = c->cache_dt == AS_BF16;
+    a.n_planes = NG;
     a.cache_lse = c->lse_planes;
     a.plane_out = L.dst_plane_out;
     a.plane_lse = L.dst_plane_lse;
@@ -544,11 +556,28 @@ as_status as_step_cp(as_cache* c, const void* q, const void* k_buf, const void* 
 }
 
 as_status as_device_status(void* stream, uint32_t* h_bits) {
-  unsigned int bits = 0;
-  cudaError_t e = asp::read_and_clear_dev_error(&bits, static_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "device status");
+  unsigned int bits = 0;
+  for (auto reader : {asp::dev_error_attn_tc, asp::dev_error_attn_simt, asp::dev_error_compose}) {
+    unsigned int b = 0;
+    if ((e = reader(&b)) != cudaSuccess) return cuda_fail(e, "device status");
+    bits |= b;
+  }
   if (h_bits) *h_bits = bits;
   if (bits & AS_DEVERR_TIMEOUT) return fail(AS_ERR_TIMEOUT, "a kernel's bounded wait ran out (bits 0x%x)", bits);
+  if (bits & AS_DEVERR_BOUNDS)
+    return fail(AS_ERR_BOUNDS, "a checked build's index check failed and skipped its access (bits 0x%x)", bits);
+  return ok();
+}
+
+as_status as_debug_bounds_probe(float* buf, int64_t n, void* stream) {
+  if (!ASP_CHECKED_BUILD) return fail(AS_ERR_UNSUPPORTED, "as_debug_bounds_probe needs the checked build (ASP_DEBUG)");
+  if (!buf || n < 0 || !aligned16(buf)) return fail(AS_ERR_INVALID_ARG, "bounds probe: bad buffer");
+  as_status s = check_device();
+  if (s != AS_OK) return s;
+  cudaError_t e = asp::launch_bounds_probe(buf, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounds probe launch");
   return ok();
 }
 
@@ -612,6 +641,7 @@ as_status as_local_states(const void* q, const void* k, const void* v, as_dtype 
   L.dst_lse = lse;
   L.dst_rows = S;
   L.dst_row0 = 0;
+  L.dst_planes = 1;
   if ((s = check_device()) != AS_OK) return s;
   if ((s = launch_attn(L, dt, static_cast<cudaStream_t>(stream))) != AS_OK) return s;
   return ok();

@@ -27,6 +27,40 @@ __device__ __forceinline__ void raise_dev_error(unsigned int bits) {
   atomicOr(&g_dev_error, bits);
 }
 
+// This translation unit's error word, read and cleared (host; the caller has
+// synchronised the work whose errors it wants).
+static inline cudaError_t read_and_clear_local_dev_error(unsigned int* bits) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return e;
+  }
+  *bits = v;
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// checked build (ASP_DEBUG=1): ASP_CHECK(cond) is cond, and when cond is false
+// it also records AS_DEVERR_BOUNDS in the device error word, so that the
+// access it guards is skipped and the host learns of it (no trap).  In the
+// normal build it is `true` and costs nothing.
+// ---------------------------------------------------------------------------
+#ifndef ASP_DEBUG
+#define ASP_DEBUG 0
+#endif
+__device__ __forceinline__ bool check_or_flag(bool ok) {
+  if (!ok) raise_dev_error(AS_DEVERR_BOUNDS);
+  return ok;
+}
+#if ASP_DEBUG
+#define ASP_CHECK(cond) (::asp::check_or_flag(static_cast<bool>(cond)))
+#else
+#define ASP_CHECK(cond) true
+#endif
+
 // ---------------------------------------------------------------------------
 // shared-memory addresses and mbarriers
 // ---------------------------------------------------------------------------

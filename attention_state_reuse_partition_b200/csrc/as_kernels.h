@@ -15,6 +15,7 @@
 
 // bits of the device error word
 #define AS_DEVERR_TIMEOUT 1u
+#define AS_DEVERR_BOUNDS 2u  // checked build (ASP_DEBUG): an index check failed and its access was skipped
 
 namespace asp {
 
@@ -46,6 +47,7 @@ struct AttnLaunch {
   void* dst_out;
   float* dst_lse;
   int dst_bf16;
+  int dst_planes;  // planes the destination holds (the checked build's bound on dest_of)
   int dst_rows, dst_row0;
   long long dst_plane_out, dst_plane_lse;
 };
@@ -70,6 +72,7 @@ struct ComposePlan {
   uint8_t nsrc[AS_MAX_P];
   const void* cache_out;  // fp32, or bf16 when cache_bf16
   int cache_bf16;
+  int n_planes;  // cache planes (the checked build's bound on src)
   const float* cache_lse;
   long long plane_out, plane_lse;
   const float* local_out;  // [B,H,S,d] local states AS(i,i) (source -2), may be null
@@ -103,6 +106,12 @@ cudaError_t launch_residual_decode(const int8_t* codes, const float* scales, voi
                                    cudaStream_t st);
 cudaError_t launch_timeout_probe(unsigned int polls, unsigned int ns, cudaStream_t st);
 cudaError_t launch_exp2_probe(const float* x, float* y, long long n, int mode, cudaStream_t st);
-cudaError_t read_and_clear_dev_error(unsigned int* bits, cudaStream_t st);
+// Each translation unit holds its own device error word (no relocatable
+// device code); each returns and clears its own.
+cudaError_t dev_error_attn_tc(unsigned int* bits);
+cudaError_t dev_error_attn_simt(unsigned int* bits);
+cudaError_t dev_error_compose(unsigned int* bits);
+// checked build only: one thread writes buf[n] behind an index check against n
+cudaError_t launch_bounds_probe(float* buf, long long n, cudaStream_t st);
 
 }  // namespace asp

@@ -86,8 +86,10 @@ __global__ void __launch_bounds__(ROWS) attn_simt_kernel(const __grid_constant__
         m = m_new;
       }
     }
-    if (s_row < q_hi) {
-      const int dest = sched.group_dest[g];
+    const int dest = sched.group_dest[g];
+    const int row0 = dest < 0 ? L.out_row0 : L.dst_row0;
+    const int rows = dest < 0 ? L.out_rows : L.dst_rows;
+    if (s_row < q_hi && ASP_CHECK(dest < L.dst_planes && s_row >= row0 && s_row < row0 + rows)) {
       float* orow;
       __nv_bfloat16* brow = nullptr;  // bf16 cache planes
       float* lrow;
@@ -127,6 +129,8 @@ cudaError_t launch_d(const AttnLaunch& L, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t dev_error_attn_simt(unsigned int* bits) { return read_and_clear_local_dev_error(bits); }
 
 cudaError_t launch_attn_simt_f32(const AttnLaunch& L, cudaStream_t st) {
   if (L.d == 128) return launch_d<128>(L, st);

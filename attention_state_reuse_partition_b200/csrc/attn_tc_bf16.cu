@@ -446,6 +446,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // the warp's 32 rows are consecutive in the destination: s_row0 + rr
         const int s_row0 = s_row - lane;
         const int dest = c.sched.group_dest[group];
+        // checked build: the destination plane and the warp's rows lie inside
+        // the destination (rows at or beyond q_hi are never written)
+        const bool in_dest = ASP_CHECK(dest < L.dst_planes &&
+                                       s_row0 >= (dest < 0 ? L.out_row0 : L.dst_row0) &&
+                                       min(s_row0 + 32, q_hi) <= (dest < 0 ? L.out_row0 + L.out_rows
+                                                                           : L.dst_row0 + L.dst_rows));
         float* orow0;  // row s_row0 (fp32 destinations)
         __nv_bfloat16* brow0 = nullptr;  // row s_row0 (bf16 cache planes)
         float* lrow;
@@ -485,7 +491,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int rr = 8 * i + rb_row;
             const float4 v4 = *reinterpret_cast<const float4*>(stage + rr * STAGE_LD + rb_col);
             const long long off = static_cast<long long>(rr) * D + ch * 16 + rb_col;
-            if (s_row0 + rr < q_hi) {
+            if (s_row0 + rr < q_hi && in_dest) {
               if (brow0)
                 *reinterpret_cast<uint2*>(brow0 + off) = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
               else
@@ -494,7 +500,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           __syncwarp();
         }
-        if (s_row < q_hi) *lrow = (m + log2f(l)) * 0.6931471805599453f;
+        if (s_row < q_hi && in_dest) *lrow = (m + log2f(l)) * 0.6931471805599453f;
       }
     }
     tc_fence_before();
@@ -592,19 +598,25 @@ cudaError_t launch_timeout_probe(unsigned int polls, unsigned int ns, cudaStream
   return cudaGetLastError();
 }
 
-cudaError_t read_and_clear_dev_error(unsigned int* bits, cudaStream_t st) {
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return e;
-  unsigned int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v));
-  if (e != cudaSuccess) return e;
-  if (v != 0) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero));
-    if (e != cudaSuccess) return e;
-  }
-  *bits = v;
-  return cudaSuccess;
+cudaError_t dev_error_attn_tc(unsigned int* bits) { return read_and_clear_local_dev_error(bits); }
+
+#if ASP_DEBUG
+__global__ void bounds_probe_kernel(float* buf, long long n) {
+  const long long idx = n;  // one past the logical end
+  if (ASP_CHECK(idx < n)) buf[idx] = 1.0f;
+}
+#endif
+
+cudaError_t launch_bounds_probe(float* buf, long long n, cudaStream_t st) {
+#if ASP_DEBUG
+  bounds_probe_kernel<<<1, 1, 0, st>>>(buf, n);
+  return cudaGetLastError();
+#else
+  (void)buf;
+  (void)n;
+  (void)st;
+  return cudaErrorNotSupported;
+#endif
 }
 
 cudaError_t launch_attn_tc_bf16(const AttnLaunch& L, cudaStream_t st) {

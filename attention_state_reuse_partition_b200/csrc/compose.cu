@@ -228,7 +228,8 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
     // source in every lane
     auto src = [&](int k) {
       const int j = list[k];
-      const long long jj = j < 0 ? 0 : j;
+      // checked build: a source is the composite, the local state or a plane of the cache
+      const long long jj = (j < 0 || !ASP_CHECK(j >= -2 && j < a.n_planes)) ? 0 : j;
       const void* o = static_cast<const E*>(a.cache_out) + jj * a.plane_out;
       const float* l = a.cache_lse + jj * a.plane_lse;
       o = j == -2 ? static_cast<const void*>(a.local_out) : o;
@@ -267,6 +268,8 @@ cudaError_t grid_for(long long nblk, unsigned* grid) {
 }
 
 }  // namespace
+
+cudaError_t dev_error_compose(unsigned int* bits) { return read_and_clear_local_dev_error(bits); }
 
 cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st) {
   const long long nblk = (a.rows + RB - 1) / RB;

@@ -47,7 +47,8 @@ typedef enum {
   AS_ERR_UNSUPPORTED = 2,  /* valid request outside the built paths */
   AS_ERR_CACHE_MISS = 3,   /* the plan reuses an entry never stored, or other members than stored */
   AS_ERR_CUDA = 4,         /* a CUDA runtime call failed (message in as_last_error) */
-  AS_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see as_device_status) */
+  AS_ERR_TIMEOUT = 5,      /* a kernel's bounded wait ran out (see as_device_status) */
+  AS_ERR_BOUNDS = 6        /* checked build only: a device index check failed (see as_device_status) */
 } as_status;
 
 typedef enum {
@@ -266,7 +267,8 @@ as_status as_residual_decode(const int8_t* codes, const float* scales, void* bas
 
 /* Synchronise `stream`, then read and clear the device error word that the
  * kernels' bounded waits set.  *h_bits receives the raw bits (may be NULL).
- * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, else AS_OK.
+ * Returns AS_ERR_TIMEOUT if a wait ran out since the last call, AS_ERR_BOUNDS
+ * if a checked build's index check failed, else AS_OK.
  *   Every wait inside the attention kernel is bounded by 1 s of the GPU's
  *   %globaltimer.  A CTA whose pipeline stops therefore gives up at most 1 s
  *   after its wait began, then waits (again at most 1 s each, three at most)
@@ -274,6 +276,22 @@ as_status as_residual_decode(const int8_t* codes, const float* scales, void* bas
  *   launch ends at most about 4 s after the stall, and this call then
  *   reports AS_ERR_TIMEOUT. */
 as_status as_device_status(void* stream, uint32_t* h_bits);
+
+/* The checked build.  `python -m attention_state_reuse_partition_b200.build`
+ * also builds libasp_debug.so with ASP_DEBUG=1 (the Python binding loads it
+ * when the environment sets ASP_DEBUG=1; as_version then ends in "checked").
+ * compute-sanitizer being closed on the GPU pool this library targets, its
+ * kernels check, before each store whose index comes from a launch's
+ * arguments, that the index lies inside its destination (the attention
+ * epilogues' destination plane and rows, the step compose's source planes);
+ * a failed check skips the access and sets a bit that as_device_status
+ * reports as AS_ERR_BOUNDS.  The normal build compiles the checks away.
+ *
+ * Test hook of the checked build: one thread writes buf[n], one past a
+ * logical length n, behind the index check, which must refuse it.  Give buf
+ * more than n floats, so that even a missing check writes inside the
+ * allocation.  AS_ERR_UNSUPPORTED in the normal build (nothing launched). */
+as_status as_debug_bounds_probe(float* buf, int64_t n, void* stream);
 
 /* Test hook for failure detection: launches one CTA that waits on a barrier
  * that nothing completes, with the kernels' wait code and a limit of

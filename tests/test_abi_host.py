@@ -471,3 +471,12 @@ def test_residual_codec_checks(api):
         assert st == _lib.AS_ERR_INVALID_ARG and frag in msg, (args, msg)
     st, msg = _status(lambda: L.as_residual_decode(p, p, p + 4, 10, 64, None))
     assert st == _lib.AS_ERR_INVALID_ARG and "aligned" in msg
+
+
+def test_checked_build_probe_needs_the_checked_library(api):
+    """The normal library refuses the bounds probe before any launch."""
+    from attention_state_reuse_partition_b200 import _lib
+    if _lib.CHECKED:
+        pytest.skip("checked library loaded")
+    st, msg = _status(lambda: _lib.LIB.as_debug_bounds_probe(1 << 20, 32, None))
+    assert st == _lib.AS_ERR_UNSUPPORTED and "checked build" in msg
