@@ -248,6 +248,140 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
   }
 }
 
+// Step compose with bf16 cache planes, all loads of a block issued at once.
+//
+// compose_rows takes one source per trip to memory (its loop branches on the
+// source's type, so the compiler does not hoist the next source's loads), and
+// with few sources per row (bf16 groups: the composite and three or four
+// planes) the warps spend their time waiting: 0.47 of HBM bandwidth.  Here a
+// warp block of BRB rows issues, before using any of them, the LSEs of every
+// source, the rows of the fp32 sources (composite, local state: at most two)
+// and the packed rows of up to PLANES_PER_TRIP bf16 planes, so one trip to
+// memory serves the whole block (a further trip per PLANES_PER_TRIP planes).
+constexpr int BRB = 4;               // rows per warp block
+constexpr int PLANES_PER_TRIP = 4;   // bf16 planes whose rows are in flight together
+
+template <int D>
+struct Packed;  // this lane's share of one bf16 row: D / 32 values
+template <>
+struct Packed<128> {
+  using T = uint2;
+  static __device__ __forceinline__ void fma(float4& a, float c, const uint2& u) {
+    a.x = fmaf(c, bf_lo(u.x), a.x);
+    a.y = fmaf(c, bf_hi(u.x), a.y);
+    a.z = fmaf(c, bf_lo(u.y), a.z);
+    a.w = fmaf(c, bf_hi(u.y), a.w);
+  }
+};
+template <>
+struct Packed<64> {
+  using T = uint32_t;
+  static __device__ __forceinline__ void fma(float2& a, float c, const uint32_t& u) {
+    a.x = fmaf(c, bf_lo(u), a.x);
+    a.y = fmaf(c, bf_hi(u), a.y);
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_bf16_kernel(const __grid_constant__ ComposePlan a) {
+  using V = Vec<D>;
+  using T = typename V::T;
+  using PK = typename Packed<D>::T;
+  const int lane = threadIdx.x & 31;
+  const int bpp = (a.n + BRB - 1) / BRB;  // warp blocks per (head, partition)
+  const long long nblk = static_cast<long long>(a.B) * a.H * a.P * bpp;
+  const long long gw = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
+  const long long stride = static_cast<long long>(gridDim.x) * WARPS;
+  for (long long b = gw; b < nblk; b += stride) {
+    const int rb = static_cast<int>(b % bpp);
+    const int i = static_cast<int>((b / bpp) % a.P);
+    const int nsrc = a.nsrc[i];
+    if (nsrc == 0) continue;  // the composite already is the final state
+    const long long bh = b / (static_cast<long long>(bpp) * a.P);
+    const int s0 = i * a.n + rb * BRB;
+    const int nr = min(BRB, (i + 1) * a.n - s0);
+    const long long row0 = bh * a.S + s0;
+    const int8_t* list = a.src[i];
+    const int nf = (list[0] < 0) + (nsrc > 1 && list[1] < 0);  // the fp32 sources lead
+    auto out_of = [&](int k) -> const void* {
+      const int j = list[k];
+      if (j == -1) return a.out;
+      if (j == -2) return a.local_out;
+      const long long jj = ASP_CHECK(j >= 0 && j < a.n_planes) ? j : 0;
+      return static_cast<const __nv_bfloat16*>(a.cache_out) + jj * a.plane_out;
+    };
+    auto lse_of = [&](int k) -> const float* {
+      const int j = list[k];
+      if (j == -1) return a.lse;
+      if (j == -2) return a.local_lse;
+      const long long jj = ASP_CHECK(j >= 0 && j < a.n_planes) ? j : 0;
+      return a.cache_lse + jj * a.plane_lse;
+    };
+    // every load of the block's first trip: LSEs (lane k: source k), fp32 rows, bf16 rows
+    float lv[BRB];
+    {
+      const float* lp = lane < nsrc ? lse_of(lane) + row0 : nullptr;
+#pragma unroll
+      for (int rr = 0; rr < BRB; ++rr) lv[rr] = (lp != nullptr && rr < nr) ? lp[rr] : -INFINITY;
+    }
+    T xf[2][BRB];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float* base = k < nf ? static_cast<const float*>(out_of(k)) + row0 * D : nullptr;
+#pragma unroll
+      for (int rr = 0; rr < BRB; ++rr)
+        xf[k][rr] = (base != nullptr && rr < nr) ? reinterpret_cast<const T*>(base + rr * D)[lane] : V::zero();
+    }
+    PK xe[PLANES_PER_TRIP][BRB];
+    auto load_planes = [&](int k0) {
+#pragma unroll
+      for (int e = 0; e < PLANES_PER_TRIP; ++e) {
+        const __nv_bfloat16* base =
+            k0 + e < nsrc ? static_cast<const __nv_bfloat16*>(out_of(k0 + e)) + row0 * D : nullptr;
+#pragma unroll
+        for (int rr = 0; rr < BRB; ++rr)
+          xe[e][rr] = (base != nullptr && rr < nr) ? reinterpret_cast<const PK*>(base + rr * D)[lane] : PK{};
+      }
+    };
+    load_planes(nf);
+    // weights: this lane's source weight per row; lane rr keeps row rr's LSE
+    float coef[BRB];
+    float lse_out = -INFINITY;
+#pragma unroll
+    for (int rr = 0; rr < BRB; ++rr) {
+      const float m = warp_max(lv[rr]);
+      const float e = m != -INFINITY ? __expf(lv[rr] - m) : 0.f;
+      const float tot = warp_sum(e);
+      coef[rr] = tot > 0.f ? e / tot : 0.f;
+      if (lane == rr && tot > 0.f) lse_out = m + __logf(tot);
+    }
+    T acc[BRB];
+#pragma unroll
+    for (int rr = 0; rr < BRB; ++rr) acc[rr] = V::zero();
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int rr = 0; rr < BRB; ++rr) {
+        const float c = __shfl_sync(0xffffffffu, coef[rr], k);
+        if (k < nf) V::fma(acc[rr], c, xf[k][rr]);
+      }
+    for (int k0 = nf; k0 < nsrc; k0 += PLANES_PER_TRIP) {
+      if (k0 > nf) load_planes(k0);
+#pragma unroll
+      for (int e = 0; e < PLANES_PER_TRIP; ++e)
+#pragma unroll
+        for (int rr = 0; rr < BRB; ++rr) {
+          const float c = __shfl_sync(0xffffffffu, coef[rr], min(k0 + e, 31));
+          if (k0 + e < nsrc) Packed<D>::fma(acc[rr], c, xe[e][rr]);
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < BRB; ++rr)
+      if (rr < nr) reinterpret_cast<T*>(a.out + (row0 + rr) * D)[lane] = acc[rr];
+    if (lane < nr) a.lse[row0 + lane] = lse_out;
+  }
+}
+
 // SMs of the current device
 cudaError_t sm_count(int* n) {
   int dev = 0;
@@ -286,6 +420,27 @@ cudaError_t launch_compose_strided(const ComposeStrided& a, cudaStream_t st) {
 }
 
 cudaError_t launch_compose_plan(const ComposePlan& a, cudaStream_t st) {
+  // bf16 planes with at most two fp32 sources and 32 sources per row: the
+  // batched kernel
+  bool batched = a.cache_bf16 != 0;
+  for (int i = 0; i < a.P && batched; ++i) {
+    int nf = 0;
+    while (nf < a.nsrc[i] && a.src[i][nf] < 0) ++nf;
+    batched = nf <= 2 && a.nsrc[i] <= 32;
+  }
+  if (batched) {
+    const long long nblk = static_cast<long long>(a.B) * a.H * a.P * ((a.n + BRB - 1) / BRB);
+    unsigned grid = 0;
+    cudaError_t e = grid_for(nblk, &grid);
+    if (e != cudaSuccess) return e;
+    if (a.d == 128)
+      compose_plan_bf16_kernel<128><<<grid, WARPS * 32, 0, st>>>(a);
+    else if (a.d == 64)
+      compose_plan_bf16_kernel<64><<<grid, WARPS * 32, 0, st>>>(a);
+    else
+      return cudaErrorInvalidValue;
+    return cudaGetLastError();
+  }
   const long long nblk = static_cast<long long>(a.B) * a.H * a.P * ((a.n + RB - 1) / RB);
   unsigned grid = 0;
   cudaError_t e = grid_for(nblk, &grid);
