@@ -258,8 +258,14 @@ __global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_kernel(const __gri
 // source, the rows of the fp32 sources (composite, local state: at most two)
 // and the packed rows of up to PLANES_PER_TRIP bf16 planes, so one trip to
 // memory serves the whole block (a further trip per PLANES_PER_TRIP planes).
+// Measured on the video reuse step with bf16 groups of 4 (ncu, per launch):
+// 2 CTAs per SM with 4 planes per trip 367 us, 4 CTAs with 2-row blocks 366,
+// 3 CTAs with 2-row blocks 412, 3 CTAs with 4-row blocks and 3 planes per
+// trip 334 (used; 32 bytes of register spill at the 85-register cap), against
+// 496 us for compose_rows.
 constexpr int BRB = 4;               // rows per warp block
-constexpr int PLANES_PER_TRIP = 4;   // bf16 planes whose rows are in flight together
+constexpr int PLANES_PER_TRIP = 3;   // bf16 planes whose rows are in flight together
+constexpr int BATCHED_CTAS_PER_SM = 3;
 
 template <int D>
 struct Packed;  // this lane's share of one bf16 row: D / 32 values
@@ -283,7 +289,8 @@ struct Packed<64> {
 };
 
 template <int D>
-__global__ void __launch_bounds__(WARPS * 32, 2) compose_plan_bf16_kernel(const __grid_constant__ ComposePlan a) {
+__global__ void __launch_bounds__(WARPS * 32, BATCHED_CTAS_PER_SM) compose_plan_bf16_kernel(
+    const __grid_constant__ ComposePlan a) {
   using V = Vec<D>;
   using T = typename V::T;
   using PK = typename Packed<D>::T;
