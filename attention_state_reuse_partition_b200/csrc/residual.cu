@@ -13,7 +13,8 @@
 // operation rounded on its own (no fused multiply-add), so the codes and the
 // reconstruction are bit-reproducible on the host.
 //
-// One warp per row, d / 32 values per lane; persistent grid.  HBM-bound:
+// One warp per row, d / 32 values per lane, four rows in flight per warp;
+// persistent grid.  HBM-bound:
 // per row the encoder reads 2 d bf16 values and writes d codes, 4 bytes of
 // scale and d bf16 values; the decoder reads d codes, the scale and d bf16
 // values and writes d bf16 values.
@@ -73,6 +74,11 @@ __device__ __forceinline__ float apply_one(float base, int q, float s) {
   return __fadd_rn(base, __fmul_rn(static_cast<float>(q), s));
 }
 
+// Each warp takes ROWS_PER_TRIP rows per iteration, their loads issued
+// before any of them is used (one row per trip left the encoder at about
+// half of HBM bandwidth, bound by latency).
+constexpr int ROWS_PER_TRIP = 4;
+
 template <int D>
 __global__ void __launch_bounds__(WARPS * 32) residual_encode_kernel(const __nv_bfloat16* __restrict__ x,
                                                                      __nv_bfloat16* __restrict__ base,
@@ -81,32 +87,48 @@ __global__ void __launch_bounds__(WARPS * 32) residual_encode_kernel(const __nv_
   constexpr int E = D / 32;
   using L = Lane<E>;
   const int lane = threadIdx.x & 31;
-  const long long stride = static_cast<long long>(gridDim.x) * WARPS;
-  for (long long row = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5); row < rows; row += stride) {
-    const long long off = row * D + lane * E;
-    float xv[E], bv[E], r[E];
-    unpack_bf16<E>(*reinterpret_cast<const typename L::B16*>(x + off), xv);
-    unpack_bf16<E>(*reinterpret_cast<const typename L::B16*>(base + off), bv);
-    float amax = 0.f;
+  const long long nw = static_cast<long long>(gridDim.x) * WARPS;
+  const long long w = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
+  for (long long r0 = w; r0 < rows; r0 += nw * ROWS_PER_TRIP) {
+    typename L::B16 xu[ROWS_PER_TRIP], bu[ROWS_PER_TRIP];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      r[e] = __fsub_rn(xv[e], bv[e]);
-      amax = fmaxf(amax, fabsf(r[e]));
+    for (int k = 0; k < ROWS_PER_TRIP; ++k) {
+      const long long row = r0 + k * nw;
+      if (row < rows) {
+        const long long off = row * D + lane * E;
+        xu[k] = *reinterpret_cast<const typename L::B16*>(x + off);
+        bu[k] = *reinterpret_cast<const typename L::B16*>(base + off);
+      }
     }
-    amax = warp_max_f(amax);
-    const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
-    const float s = __fdiv_rn(amax, 127.f);
-    typename L::Q8 qp = 0;
-    float nb[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int q = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(r[e], inv)), -127.f), 127.f));
-      qp |= static_cast<typename L::Q8>(static_cast<uint8_t>(static_cast<int8_t>(q))) << (8 * e);
-      nb[e] = apply_one(bv[e], q, s);
+    for (int k = 0; k < ROWS_PER_TRIP; ++k) {
+      const long long row = r0 + k * nw;
+      if (row >= rows) break;
+      const long long off = row * D + lane * E;
+      float xv[E], bv[E], r[E];
+      unpack_bf16<E>(xu[k], xv);
+      unpack_bf16<E>(bu[k], bv);
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        r[e] = __fsub_rn(xv[e], bv[e]);
+        amax = fmaxf(amax, fabsf(r[e]));
+      }
+      amax = warp_max_f(amax);
+      const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+      const float s = __fdiv_rn(amax, 127.f);
+      typename L::Q8 qp = 0;
+      float nb[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int q = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(r[e], inv)), -127.f), 127.f));
+        qp |= static_cast<typename L::Q8>(static_cast<uint8_t>(static_cast<int8_t>(q))) << (8 * e);
+        nb[e] = apply_one(bv[e], q, s);
+      }
+      *reinterpret_cast<typename L::Q8*>(codes + off) = qp;
+      *reinterpret_cast<typename L::B16*>(base + off) = pack_bf16<E>(nb);
+      if (lane == 0) scales[row] = s;
     }
-    *reinterpret_cast<typename L::Q8*>(codes + off) = qp;
-    *reinterpret_cast<typename L::B16*>(base + off) = pack_bf16<E>(nb);
-    if (lane == 0) scales[row] = s;
   }
 }
 
@@ -118,19 +140,36 @@ __global__ void __launch_bounds__(WARPS * 32) residual_decode_kernel(const int8_
   constexpr int E = D / 32;
   using L = Lane<E>;
   const int lane = threadIdx.x & 31;
-  const long long stride = static_cast<long long>(gridDim.x) * WARPS;
-  for (long long row = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5); row < rows; row += stride) {
-    const long long off = row * D + lane * E;
-    const float s = scales[row];
-    const typename L::Q8 qp = *reinterpret_cast<const typename L::Q8*>(codes + off);
-    float bv[E], nb[E];
-    unpack_bf16<E>(*reinterpret_cast<const typename L::B16*>(base + off), bv);
+  const long long nw = static_cast<long long>(gridDim.x) * WARPS;
+  const long long w = static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
+  for (long long r0 = w; r0 < rows; r0 += nw * ROWS_PER_TRIP) {
+    typename L::Q8 qu[ROWS_PER_TRIP];
+    typename L::B16 bu[ROWS_PER_TRIP];
+    float su[ROWS_PER_TRIP];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int q = static_cast<int8_t>(static_cast<uint8_t>(qp >> (8 * e)));
-      nb[e] = apply_one(bv[e], q, s);
+    for (int k = 0; k < ROWS_PER_TRIP; ++k) {
+      const long long row = r0 + k * nw;
+      if (row < rows) {
+        const long long off = row * D + lane * E;
+        qu[k] = *reinterpret_cast<const typename L::Q8*>(codes + off);
+        bu[k] = *reinterpret_cast<const typename L::B16*>(base + off);
+        su[k] = scales[row];
+      }
     }
-    *reinterpret_cast<typename L::B16*>(base + off) = pack_bf16<E>(nb);
+#pragma unroll
+    for (int k = 0; k < ROWS_PER_TRIP; ++k) {
+      const long long row = r0 + k * nw;
+      if (row >= rows) break;
+      const long long off = row * D + lane * E;
+      float bv[E], nb[E];
+      unpack_bf16<E>(bu[k], bv);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int q = static_cast<int8_t>(static_cast<uint8_t>(qu[k] >> (8 * e)));
+        nb[e] = apply_one(bv[e], q, su[k]);
+      }
+      *reinterpret_cast<typename L::B16*>(base + off) = pack_bf16<E>(nb);
+    }
   }
 }
 
@@ -140,7 +179,7 @@ cudaError_t grid_for_rows(long long rows, unsigned* grid) {
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const long long ctas = (rows + WARPS - 1) / WARPS;
+  const long long ctas = (rows + WARPS * ROWS_PER_TRIP - 1) / (WARPS * ROWS_PER_TRIP);
   const long long cap = static_cast<long long>(sms) * CTAS_PER_SM;
   *grid = static_cast<unsigned>(ctas < cap ? (ctas > 0 ? ctas : 1) : cap);
   return cudaSuccess;
