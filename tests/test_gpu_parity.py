@@ -186,6 +186,36 @@ def test_attn_bf16_flux_full(api):
     check_bf16(out[:, heads][:, :, rows], lse[:, heads][:, :, rows], ref_o, ref_l, "flux_image sampled rows")
 
 
+@pytest.mark.parametrize("H,S,P,d", [(96, 512, 4, 128), (200, 128, 1, 64), (80, 640, 5, 128)])
+def test_attn_bf16_many_heads(api, H, S, P, d):
+    """More 256-row CTAs than SMs over many heads: one KV tile per CTA
+    (S = 128), a ragged last row block (S = 640: 2.5 blocks of 256 rows per
+    head), and one state per KV partition (several accumulation groups per
+    CTA)."""
+    s = W.spec("flux_image", B=1, H=H, S=S, d=d, P=P)
+    q, k, v = W.flux_qkv(s)
+    qc, kc, vc = (x.cuda() for x in (q, k, v))
+    heads = [0, 1, H // 2, H - 2, H - 1]
+    qn, kn, vn = (f64(x[:, heads]) for x in (q, k, v))
+    out, lse = api.as_partition_attn(qc, kc, vc, P, -1, list(range(P)), compose=True)
+    full_o, full_l = O.full_attention(qn, kn, vn, s.scale)
+    check_bf16(out[:, heads], lse[:, heads], full_o, full_l, f"composite H={H} S={S}")
+    po, pl = api.as_partition_attn(qc, kc, vc, P, -1, list(range(P)), compose=False)
+    ref = O.partition_states(qn, kn, vn, s.scale, P)
+    for j in range(P):
+        check_bf16(po[j][:, heads], pl[j][:, heads], ref[j][0], ref[j][1], f"partition {j} H={H} S={S}")
+
+
+def test_step_store_then_reuse_many_heads(api):
+    """An anchor step that stores every pair (one accumulation group per KV
+    partition, the same for every query partition, so one launch block of all
+    rows), then a step that reuses every stored entry, over 96 heads."""
+    s = W.spec("flux_image", B=1, H=96, S=512, P=4)
+    q, k, v = (x.cuda() for x in W.flux_qkv(s))
+    plans = [np.full((4, 4), 2, np.uint8), np.zeros((4, 4), np.uint8)]
+    _run_steps(api, s, [(q, k, v), (q, k, v)], plans, heads=[0, 47, 95])
+
+
 # ---------------------------------------------------------------------------
 # steps under a compute/reuse plan
 # ---------------------------------------------------------------------------
