@@ -358,14 +358,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc_fence_after();
       float s[BN];
       {
-        uint32_t r[4][32];
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld32(t_lane + s_col + ch * 32, r[ch]);
+        uint32_t r[128];
+        tmem_ld128(t_lane + s_col, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[ch * 32 + e] = __uint_as_float(r[ch][e]);
+        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(r[e]);
       }
       if (nv < BN) {
 #pragma unroll
@@ -415,8 +412,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // the previous PV of this tile has completed (see the header), so P may
       // be written over S and O rescaled now; P goes first, which frees its
       // registers for the rescale
-      tmem_st32(t_lane + s_col, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(t_lane + s_col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_st64(t_lane + s_col, pk);
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int ch = 0; ch < D / 16; ++ch) {
