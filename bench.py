@@ -710,6 +710,55 @@ def run_video_long(args, device, g=1, cache_dtype="f32", peaks=None, with_oracle
     return res, (orc.summary(name) if orc is not None else None)
 
 
+def run_cp(args, device, world=4):
+    """One rank after another of a context-parallel split of the long video
+    trajectory (DiTango review page, Referee Report "Summary": group-wise KV
+    transfer; each rank owns a run of query partitions, its cache entries and
+    the K/V rows it must compute fresh), on this one GPU: each rank's
+    as_step_cp over its Q rows and the compact K/V buffer the exchange would
+    give it (gathered here outside the timed region), timed with CUDA events.
+    The exchange itself needs several GPUs; its bytes come from the plan
+    (per-pair entries: reused pairs move nothing) and, with residual
+    compression, from the codec's 132 bytes per 256-byte row."""
+    from attention_state_reuse_partition_b200 import api, cp
+    heads = getattr(args, "video_heads", None)
+    s = W.spec("video_long") if heads is None else W.spec("video_long", H=heads)
+    n = s.n
+    layout = cp.CpLayout(s.P, world)
+    caches = [api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, q_first=layout.parts(r).start,
+                          q_count=len(layout.parts(r))) for r in range(world)]
+    per_step = []
+    for t, q, k, v in W.video_trajectory(s, device=device):
+        plan = W.grouped_plan_for_step(s, t, 1).numpy()
+        ms = []
+        for r in range(world):
+            mine = layout.parts(r)
+            rows = slice(mine.start * n, mine.stop * n)
+            k_buf, v_buf, slots = cp.gather_kv_local(k, v, cp.needed_kv(plan, mine), n)
+            q_r = q[:, :, rows].contiguous()
+            out = torch.empty((s.B, s.H, len(mine) * n, s.d), device=device)
+            lse = torch.empty((s.B, s.H, len(mine) * n), device=device)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            api.as_step_cp(caches[r], q_r, k_buf, v_buf, slots, plan, t, out=out, lse=lse)
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(round(a.elapsed_time(b), 3))
+            del k_buf, v_buf, q_r, out, lse
+        xb = cp.exchange_bytes(plan, layout, s.B, s.H, n, s.d, 2)
+        per_step.append({"step": t, "rank_ms": ms, "max_rank_ms": max(ms), "sum_rank_ms": round(sum(ms), 3),
+                         "balance": round(sum(ms) / (world * max(ms)), 4),
+                         "exchange_bytes": xb["moved"], "all_gather_bytes": xb["all_gather"],
+                         "exchange_bytes_residual_coded": int(xb["moved"] * 132 / 256)})
+    del caches
+    torch.cuda.empty_cache()
+    return {"workload": f"video_long (B=1 H={s.H} S={s.S} P={s.P}, window {s.window}, 4 steps), fp32 pair "
+                        f"entries, split over {world} ranks of {s.P // world} query partitions",
+            "timing": "each rank's as_step_cp alone on this GPU (CUDA events); the exchange is not run",
+            "steps": per_step}
+
+
 def run_planner(args, device, window=2, reuse_ratio=0.7, eps_local=0.5, g=1, cache_dtype="f32"):
     """Long video trajectory with the anchor-guided planner choosing each
     step's plan: local states, drift, selection, the step (which composes the
@@ -768,7 +817,7 @@ def main():
     ap.add_argument("--warm-seconds", type=float, default=1.0,
                     help="minimum duration of the warm-up (clocks settle; the sampler runs throughout)")
     ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner",
-                                       "planner_grouped", "boundary", "locality", "residual"], default=None,
+                                       "planner_grouped", "boundary", "locality", "residual", "cp"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
@@ -808,7 +857,8 @@ def main():
               "planner_grouped": lambda a, dev: run_planner(a, dev, g=4, cache_dtype="bf16"),
               "boundary": lambda a, dev: run_boundary(a, dev, float("nan")),
               "residual": lambda a, dev: run_residual(a, dev, peaks),
-              "locality": run_locality}[args.only]
+              "locality": run_locality,
+              "cp": run_cp}[args.only]
         print(json.dumps({"only": args.only, **fn(args, device)}))
         return
     if world > 1:
@@ -852,6 +902,7 @@ def main():
         roofline["partition_boundary"] = run_boundary(args, device, achieved)
         roofline["residual_codec"] = run_residual(args, device, peaks)
         roofline["locality"] = run_locality(args, device)
+        roofline["context_parallel"] = run_cp(args, device)
     if cpu is not None and legs:
         cpu["legs"] = {k: v for k, v in legs.items() if v is not None}
 
