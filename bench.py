@@ -710,7 +710,7 @@ def run_video_long(args, device, g=1, cache_dtype="f32", peaks=None, with_oracle
     return res, (orc.summary(name) if orc is not None else None)
 
 
-def run_cp(args, device, world=4):
+def run_cp(args, device, world=None):
     """One rank after another of a context-parallel split of the long video
     trajectory (DiTango review page, Referee Report "Summary": group-wise KV
     transfer; each rank owns a run of query partitions, its cache entries and
@@ -721,10 +721,22 @@ def run_cp(args, device, world=4):
     (per-pair entries: reused pairs move nothing) and, with residual
     compression, from the codec's 132 bytes per 256-byte row."""
     from attention_state_reuse_partition_b200 import api, cp
+    world = world or getattr(args, "cp_world", 4)
     heads = getattr(args, "video_heads", None)
     s = W.spec("video_long") if heads is None else W.spec("video_long", H=heads)
     n = s.n
     layout = cp.CpLayout(s.P, world)
+    # one untimed small rank step first, so that no rank pays the process's
+    # first launches
+    sw = W.spec("video_long", H=2, rows=8, cols=16, S=16 * 8 * 16)
+    lw = cp.CpLayout(sw.P, world)
+    _, qw, kw, vw = next(iter(W.video_trajectory(sw, device=device)))
+    pw = W.grouped_plan_for_step(sw, 0, 1).numpy()
+    cw = api.AsCache(sw.B, sw.H, sw.S, sw.d, sw.P, device=device, q_first=0, q_count=len(lw.parts(0)))
+    kb, vb, sl = cp.gather_kv_local(kw, vw, cp.needed_kv(pw, lw.parts(0)), sw.n)
+    api.as_step_cp(cw, qw[:, :, :len(lw.parts(0)) * sw.n].contiguous(), kb, vb, sl, pw, 0)
+    torch.cuda.synchronize()
+    del cw, kb, vb, qw, kw, vw
     caches = [api.AsCache(s.B, s.H, s.S, s.d, s.P, device=device, q_first=layout.parts(r).start,
                           q_count=len(layout.parts(r))) for r in range(world)]
     per_step = []
@@ -819,6 +831,7 @@ def main():
     ap.add_argument("--only", choices=["compose", "reuse", "video_long", "video_long_grouped", "planner",
                                        "planner_grouped", "boundary", "locality", "residual", "cp"], default=None,
                     help="run one secondary workload alone and print its JSON (for profiling)")
+    ap.add_argument("--cp-world", type=int, default=4, help="ranks of the context-parallel leg (default 4)")
     ap.add_argument("--compose-rows", type=int, default=None,
                     help="rows of the compose workload (default: all B*H*S rows)")
     ap.add_argument("--reuse-heads", type=int, default=None, help="heads of the reuse workload (default 24)")
