@@ -146,6 +146,34 @@ def test_layout_and_exchange_plan():
     assert b["moved"] == 2 * (2 * 1 * 2 * 4 * 8 * 2) and b["all_gather"] == 6 * (2 * 1 * 2 * 4 * 8 * 2)
 
 
+def test_exchange_share_on_the_long_trajectory():
+    """The exchange's share of an all-gather on the long-trajectory plans
+    (P = 32, window 4, 10% of the far pairs forced fresh each step): the
+    anchor moves everything, and a reuse step moves, at 2, 4 and 8 ranks,
+    0.72-0.91, 0.64-0.75 and 0.48-0.52 of an all-gather.  The window alone
+    (no forced pairs) moves 0.25 at each size: every rank receives the 4
+    partitions on either side of its run."""
+    from attention_state_reuse_partition_b200 import cp
+    from attention_state_reuse_partition_b200 import workloads as W
+    s = W.spec("video_long")
+    bounds = {2: (0.71, 0.91), 4: (0.63, 0.75), 8: (0.48, 0.52)}
+    for world, (lo, hi) in bounds.items():
+        lay = cp.CpLayout(s.P, world)
+        for t in range(s.steps):
+            b = cp.exchange_bytes(W.grouped_plan_for_step(s, t, 1).numpy(), lay, s.B, s.H, s.n, s.d, 2)
+            share = b["moved"] / b["all_gather"]
+            if t == 0:
+                assert share == 1.0
+            else:
+                assert lo <= share <= hi, (world, t, share)
+        window = np.array([[1 if abs(i - j) <= s.window else 0 for j in range(s.P)] for i in range(s.P)], np.uint8)
+        b = cp.exchange_bytes(window, lay, s.B, s.H, s.n, s.d, 2)
+        # rank r receives the partitions within `window` of its run that other ranks own
+        want = sum(len([j for j in range(s.P) if j not in lay.parts(r)
+                        and min(abs(j - i) for i in lay.parts(r)) <= s.window]) for r in range(world))
+        assert b["moved"] == want * 2 * s.B * s.H * s.n * s.d * 2
+
+
 class _OracleCodec:
     """The oracle's residual coding on CPU tensors (float32 holding bf16
     values), for the host logic of the residual exchange."""
